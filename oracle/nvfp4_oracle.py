@@ -1,0 +1,319 @@
+"""CPU oracle for the NVFP4 block-scaled GEMM with a fused BF16 LoRA correction.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this module.
+The product path (the CUDA library and its Python binding) never imports, links or
+calls anything here, and this module imports nothing from the product.
+
+It restates, slowly and in float64, what the pages define:
+
+* ``flashinfer.gemm.mm_nvfp4_lora`` -- opening formula
+  ``out = alpha * (dequant(a) @ dequant(b)^T) + lora_scale * (d @ lora_b^T) [+ bias]``,
+  the paragraph after it (operands consumed as ``mm_fp4`` does: E2M1 codes packed two
+  per byte, UE4M3 scales over 16 K-elements in the 128x4 swizzled layout; correction
+  in fp32 in the same kernel; one rounding to bf16), the "Raw path" and "Prepared path"
+  bullets, and the Parameters entries for a, b, a_sf, b_sf, alpha, d, lora_b,
+  lora_scale and bias.
+* ``flashinfer.gemm.prepare_nvfp4_lora_adapter`` -- summary paragraph (the fold:
+  ``ratio = div.rn.f32(lora_scale, alpha[0])``,
+  ``b_folded[i] = bf16_rne(fp32(lora_b[i]) * ratio)``).
+
+Readings taken where the pages are silent (each is listed in the design doc):
+
+* nibble order: element ``2j`` of a row is the LOW nibble of byte ``j``.  The GEMM
+  result does not depend on it (both nibbles of a byte sit in the same 16-block and
+  A and B use the same convention), only generators do;
+* the 128x4 swizzle is the block-scale layout of the tensor-core scale copy:
+  ``offset(r, c) = ((r // 128) * (C // 4) + c // 4) * 512 + (r % 32) * 16
+  + ((r % 128) // 32) * 4 + (c % 4)`` with ``C = K // 16`` scale columns;
+* UE4M3 byte ``0x7F`` is NaN; a byte with bit 7 set is not a UE4M3 value and is
+  rejected;
+* the output rounding goes from the float64 value straight to bf16 (round to nearest,
+  ties to even, subnormals kept, overflow to infinity) -- one rounding, no float32 step;
+* raw epilogue ``alpha*base + s*L (+ bias)``; prepared ``alpha*(base + L_folded)
+  (+ bias)`` (bias is not multiplied by alpha); adapter-off ``alpha*base (+ bias)``;
+* NaN produced by the fold is stored as 0x7FC0, PyTorch's bf16 NaN.
+
+Parity of the base product: with the configs' scale range every product
+``e2m1 * e2m1 * ue4m3 * ue4m3`` is a multiple of 2**-12 below 576 in magnitude, so
+partial sums over K <= 8192 need at most 35 significant bits and the float64 matmul
+below is exact whatever order the library sums in.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+# --------------------------------------------------------------------------------------
+# Element formats (mm_nvfp4_lora page, paragraph after the formula and Parameters: a, b,
+# a_sf, b_sf).  The pages name the formats; their value sets are fixed by the formats.
+# --------------------------------------------------------------------------------------
+
+#: E2M1 value of each 4-bit code (bit 3 sign, bits 2..1 exponent with bias 1, bit 0
+#: mantissa).  Written out as the 16-entry table.
+E2M1_TABLE = np.array(
+    [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,
+     -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0],
+    dtype=np.float64,
+)
+
+SF_VEC = 16          # K-elements covered by one UE4M3 scale
+SF_ATOM_ROWS = 128   # rows of one swizzle atom
+SF_ATOM_COLS = 4     # scale columns of one swizzle atom
+SF_ATOM_BYTES = SF_ATOM_ROWS * SF_ATOM_COLS
+
+
+def decode_e2m1(packed: np.ndarray) -> np.ndarray:
+    """Unpack ``uint8 [R, K/2]`` into float64 ``[R, K]``; element 2j = low nibble of byte j."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    lo = E2M1_TABLE[packed & 0x0F]
+    hi = E2M1_TABLE[packed >> 4]
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.float64)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def decode_ue4m3(x: np.ndarray) -> np.ndarray:
+    """UE4M3 bytes -> float64: 4 exponent bits (bias 7), 3 mantissa bits, no sign.
+
+    ``e == 0`` is subnormal (``m * 2**-9``); ``0x7F`` is NaN; max finite ``0x7E`` = 448.
+    """
+    x = np.asarray(x, dtype=np.uint8)
+    if np.any(x & 0x80):
+        raise ValueError("UE4M3 byte with bit 7 set: not an unsigned E4M3 value")
+    e = (x >> 3).astype(np.int64) & 0xF
+    m = (x & 0x7).astype(np.float64)
+    normal = (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64))
+    sub = m * 2.0 ** -9
+    val = np.where(e == 0, sub, normal)
+    return np.where(x == 0x7F, np.nan, val)
+
+
+# --------------------------------------------------------------------------------------
+# 128x4 swizzled scale layout (mm_nvfp4_lora page, Parameters: a_sf / b_sf: "128x4
+# swizzled layout (rows padded to 128); larger contiguous backing buffers are accepted")
+# --------------------------------------------------------------------------------------
+
+def padded_rows(rows: int) -> int:
+    return -(-rows // SF_ATOM_ROWS) * SF_ATOM_ROWS
+
+
+def sf_buffer_bytes(rows: int, k: int) -> int:
+    """Minimum byte size of a swizzled scale buffer for ``rows`` rows and K = ``k``."""
+    return padded_rows(rows) * (k // SF_VEC)
+
+
+def sf_offset(r, c, k: int):
+    """Byte offset of logical scale ``(row r, scale column c)`` for K = ``k``."""
+    r = np.asarray(r, dtype=np.int64)
+    c = np.asarray(c, dtype=np.int64)
+    col_atoms = (k // SF_VEC) // SF_ATOM_COLS
+    return (((r // 128) * col_atoms + c // 4) * SF_ATOM_BYTES
+            + (r % 32) * 16 + ((r % 128) // 32) * 4 + (c % 4))
+
+
+def unswizzle_scales(buf: np.ndarray, rows: int, k: int) -> np.ndarray:
+    """Logical ``uint8 [rows, k/16]`` scale matrix read out of a swizzled buffer."""
+    buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    need = sf_buffer_bytes(rows, k)
+    if buf.size < need:
+        raise ValueError(f"scale buffer has {buf.size} bytes, needs {need}")
+    rr, cc = np.meshgrid(np.arange(rows), np.arange(k // SF_VEC), indexing="ij")
+    return buf[sf_offset(rr, cc, k)]
+
+
+def swizzle_scales(logical: np.ndarray, k: int, pad_value: int = 0) -> np.ndarray:
+    """Inverse of :func:`unswizzle_scales`: place ``[rows, k/16]`` into a padded buffer."""
+    logical = np.asarray(logical, dtype=np.uint8)
+    rows = logical.shape[0]
+    buf = np.full(sf_buffer_bytes(rows, k), pad_value, dtype=np.uint8)
+    rr, cc = np.meshgrid(np.arange(rows), np.arange(k // SF_VEC), indexing="ij")
+    buf[sf_offset(rr, cc, k)] = logical
+    return buf
+
+
+def dequant(codes: np.ndarray, sf_buf: np.ndarray, rows: int, k: int) -> np.ndarray:
+    """``dequant(x)`` of the opening formula: E2M1 value times its block's UE4M3 scale."""
+    vals = decode_e2m1(np.asarray(codes, dtype=np.uint8).reshape(rows, k // 2))
+    scales = decode_ue4m3(unswizzle_scales(sf_buf, rows, k))
+    return vals * np.repeat(scales, SF_VEC, axis=1)
+
+
+# --------------------------------------------------------------------------------------
+# bf16 helpers (the output dtype; d, lora_b, bias, b_folded are bf16 bit patterns)
+# --------------------------------------------------------------------------------------
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16_rne(y: np.ndarray) -> np.ndarray:
+    """Round float64 straight to bf16 bits: nearest, ties to even, one rounding.
+
+    bf16 keeps 8 significant bits and float32's exponent range (normal down to 2**-126,
+    subnormal quantum 2**-133).  The quantum of |y| in [2**(E-1), 2**E) is
+    ``2**(max(E, -125) - 8)``; dividing by a power of two is exact, ``rint`` rounds
+    half to even, and a result of 2**128 or more is infinity.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    out = np.zeros(y.shape, dtype=np.uint16)
+    sign = np.signbit(y)
+    mag = np.abs(y)
+    finite = np.isfinite(y)
+    nz = finite & (mag > 0)
+    _, exp = np.frexp(np.where(nz, mag, 1.0))          # mag = f * 2**exp, f in [0.5, 1)
+    q_exp = np.maximum(exp, -125) - 8
+    q = np.exp2(q_exp.astype(np.float64))
+    rounded = np.rint(np.where(nz, mag, 0.0) / q) * q
+    overflow = nz & (rounded >= 2.0 ** 128)
+    fin_bits = (np.where(overflow, 0.0, rounded).astype(np.float32).view(np.uint32) >> 16)
+    out[:] = fin_bits.astype(np.uint16)
+    out[overflow] = 0x7F80
+    out[np.isinf(y)] = 0x7F80
+    out = np.where(sign, out | 0x8000, out).astype(np.uint16)
+    out[np.isnan(y)] = 0x7FC0
+    return out
+
+
+def f32_to_bf16_rne(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bits, nearest-even, NaN -> 0x7FC0 (PyTorch's bf16 NaN)."""
+    x = np.asarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    out = (rounded & 0xFFFF).astype(np.uint16)
+    out[np.isnan(x)] = 0x7FC0
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# The operation (mm_nvfp4_lora page)
+# --------------------------------------------------------------------------------------
+
+def base_product(a, b, a_sf, b_sf, M: int, N: int, K: int) -> np.ndarray:
+    """``dequant(a) @ dequant(b)^T`` in float64 (opening formula); a library matmul."""
+    return dequant(a, a_sf, M, K) @ dequant(b, b_sf, N, K).T
+
+
+def base_element(a, b, a_sf, b_sf, M: int, N: int, K: int, m: int, n: int) -> float:
+    """One element of the base product, summed block by block in float64."""
+    a_row = decode_e2m1(np.asarray(a, dtype=np.uint8).reshape(M, K // 2)[m])
+    b_row = decode_e2m1(np.asarray(b, dtype=np.uint8).reshape(N, K // 2)[n])
+    cols = np.arange(K // SF_VEC)
+    sa = decode_ue4m3(np.asarray(a_sf, dtype=np.uint8).reshape(-1)[sf_offset(m, cols, K)])
+    sb = decode_ue4m3(np.asarray(b_sf, dtype=np.uint8).reshape(-1)[sf_offset(n, cols, K)])
+    total = 0.0
+    for blk in range(K // SF_VEC):
+        sl = slice(blk * SF_VEC, (blk + 1) * SF_VEC)
+        total += float(np.dot(a_row[sl], b_row[sl])) * float(sa[blk]) * float(sb[blk])
+    return total
+
+
+def lora_term(d_bits, lb_bits, M: int, N: int, r: int) -> np.ndarray:
+    """``d @ lora_b^T`` in float64 (bf16 x bf16 products are exact in float64)."""
+    d = bf16_bits_to_f64(np.asarray(d_bits).reshape(M, r))
+    lb = bf16_bits_to_f64(np.asarray(lb_bits).reshape(N, r))
+    return d @ lb.T
+
+
+def _bias_row(bias_bits, N: int):
+    if bias_bits is None:
+        return 0.0
+    return bf16_bits_to_f64(np.asarray(bias_bits).reshape(N))[None, :]
+
+
+def mm_raw(a, b, a_sf, b_sf, alpha: float, d_bits, lb_bits, lora_scale, bias_bits,
+           M: int, N: int, K: int, r: int, base: np.ndarray | None = None) -> np.ndarray:
+    """Raw path ("Raw path" bullet): ``alpha*base + s*(d @ lora_b^T) [+ bias]``, float64.
+
+    ``lora_scale`` None or equal to zero is the zero-adapter call (Parameters:
+    lora_scale): the LoRA term is not evaluated at all.
+    """
+    if base is None:
+        base = base_product(a, b, a_sf, b_sf, M, N, K)
+    y = np.float64(alpha) * base
+    if lora_scale is not None and float(lora_scale) != 0.0:
+        y = y + np.float64(lora_scale) * lora_term(d_bits, lb_bits, M, N, r)
+    return y + _bias_row(bias_bits, N)
+
+
+def mm_prepared(a, b, a_sf, b_sf, alpha: float, d_bits, b_folded_bits, ratio, bias_bits,
+                M: int, N: int, K: int, r: int, base: np.ndarray | None = None) -> np.ndarray:
+    """Prepared path ("Prepared path" bullet): base first, LoRA with ``b_folded`` into the
+    same accumulator, alpha applied once: ``alpha*(base + d @ b_folded^T) [+ bias]``.
+
+    ``ratio`` is the fold's ``lora_scale / alpha``; a zero ratio is the zero adapter
+    (Parameters: lora_adapter -- "lora_scale == 0 produces the adapter-off output").
+    """
+    if base is None:
+        base = base_product(a, b, a_sf, b_sf, M, N, K)
+    acc = base
+    if float(ratio) != 0.0:
+        acc = acc + lora_term(d_bits, b_folded_bits, M, N, r)
+    return np.float64(alpha) * acc + _bias_row(bias_bits, N)
+
+
+def mm_off(a, b, a_sf, b_sf, alpha: float, bias_bits, M: int, N: int, K: int,
+           base: np.ndarray | None = None) -> np.ndarray:
+    """Adapter-off call (neither form): ``alpha*base [+ bias]``."""
+    if base is None:
+        base = base_product(a, b, a_sf, b_sf, M, N, K)
+    return np.float64(alpha) * base + _bias_row(bias_bits, N)
+
+
+def round_output(y: np.ndarray) -> np.ndarray:
+    """The single rounding of the fp32 result to bf16, taken here from float64."""
+    return f64_to_bf16_rne(y)
+
+
+# --------------------------------------------------------------------------------------
+# The fold (prepare_nvfp4_lora_adapter page, summary paragraph)
+# --------------------------------------------------------------------------------------
+
+def fold_ratio(lora_scale: float, alpha: float) -> np.float32:
+    """``div.rn.f32(fp32(lora_scale), fp32(alpha[0]))``: one IEEE binary32 division."""
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return np.float32(lora_scale) / np.float32(alpha)
+
+
+def fold(lb_bits, lora_scale: float, alpha: float):
+    """Return ``(ratio, b_folded_bits)``: ``b_folded[i] = bf16_rne(fp32(lora_b[i]) * ratio)``.
+
+    The product is one binary32 multiply; the rounding is nearest-even with NaN stored
+    as 0x7FC0.
+    """
+    ratio = fold_ratio(lora_scale, alpha)
+    lb32 = bf16_bits_to_f64(lb_bits).astype(np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        prod = lb32 * ratio
+    return ratio, f32_to_bf16_rne(prod.astype(np.float32))
+
+
+def eager_prepare_check(lora_scale: float, alpha: float) -> None:
+    """The eager prepare's checks (prepare_nvfp4_lora_adapter page, Parameters: alpha and
+    Returns): alpha == 0 is refused and the ratio must be finite; ValueError otherwise."""
+    if np.float32(alpha) == 0.0:
+        raise ValueError("alpha == 0: lora_scale / alpha is undefined")
+    if not np.isfinite(fold_ratio(lora_scale, alpha)):
+        raise ValueError("lora_scale / alpha is not finite")
+
+
+# --------------------------------------------------------------------------------------
+# Acceptance measures
+# --------------------------------------------------------------------------------------
+
+def tolerance(y_ref: np.ndarray) -> np.ndarray:
+    """Per-element bound ``2**-7*|ref| + 2**-10*max|ref|`` on ``|gpu - ref|``."""
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    return 2.0 ** -7 * np.abs(y_ref) + 2.0 ** -10 * np.max(np.abs(y_ref))
+
+
+def sqnr_db(y_ref: np.ndarray, y_test: np.ndarray) -> float:
+    """``10*log10(sum(ref**2) / sum((test - ref)**2))``; infinite when they agree."""
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    err = np.sum((np.asarray(y_test, dtype=np.float64) - y_ref) ** 2)
+    sig = np.sum(y_ref ** 2)
+    if err == 0.0:
+        return float("inf")
+    return float(10.0 * np.log10(sig / err))

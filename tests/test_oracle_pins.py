@@ -1,0 +1,381 @@
+"""Pins of the CPU oracle against what the formats, the pages and mathematics fix.
+
+None of these re-types the oracle's formulas: each expected value comes from a
+different route (a library decoder, a closed form written from the format
+definition, a brute-force loop, a second formulation of the layout, or an invariant),
+chosen so that a dropped term, a wrong sign or index, a swapped nibble or a
+transposed operand in the oracle fails at least one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------------------------------
+# independent decoders used only by the tests
+# ---------------------------------------------------------------------------------------
+
+def e2m1_closed_form(code: int) -> float:
+    """E2M1 from its bit fields: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0."""
+    s = -1.0 if code & 8 else 1.0
+    e = (code >> 1) & 3
+    m = code & 1
+    if e == 0:
+        return s * 0.5 * m
+    return s * (2.0 ** (e - 1)) * (1.0 + 0.5 * m)
+
+
+def ue4m3_library(byte_values) -> np.ndarray:
+    """UE4M3 through PyTorch's float8_e4m3fn decoder (bit 7 = sign = 0)."""
+    t = torch.tensor(np.asarray(byte_values, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.float().numpy().astype(np.float64)
+
+
+def swizzle_by_permute(logical: np.ndarray, k: int) -> np.ndarray:
+    """128x4 layout as a reshape/permute of the padded logical matrix:
+    [R/128, 4, 32, C/4, 4] -> [R/128, C/4, 32, 4, 4]."""
+    rows, c = logical.shape
+    rp = -(-rows // 128) * 128
+    pad = torch.zeros((rp, c), dtype=torch.uint8)
+    pad[:rows] = torch.from_numpy(logical)
+    v = pad.view(rp // 128, 4, 32, c // 4, 4).permute(0, 3, 2, 1, 4).contiguous()
+    return v.view(-1).numpy()
+
+
+def brute_base(a, b, a_sf_logical, b_sf_logical, M, N, K):
+    """Pure-Python triple loop with the closed-form decoders above."""
+    out = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for kk in range(K):
+                ab = int(a[m, kk // 2]); bb = int(b[n, kk // 2])
+                ca = (ab >> 4) if kk % 2 else (ab & 15)
+                cb = (bb >> 4) if kk % 2 else (bb & 15)
+                sa = ue4m3_library([a_sf_logical[m, kk // 16]])[0]
+                sb = ue4m3_library([b_sf_logical[n, kk // 16]])[0]
+                acc += e2m1_closed_form(ca) * e2m1_closed_form(cb) * sa * sb
+            out[m, n] = acc
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# formats
+# ---------------------------------------------------------------------------------------
+
+def test_e2m1_table_matches_bit_fields():
+    for code in range(16):
+        got = O.E2M1_TABLE[code]
+        want = e2m1_closed_form(code)
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), code
+    # negation symmetry: flipping the sign bit negates
+    for code in range(8):
+        assert O.E2M1_TABLE[code ^ 8] == -O.E2M1_TABLE[code]
+
+
+def test_e2m1_nibble_order_low_first():
+    packed = np.array([[0x71, 0x0F]], dtype=np.uint8)   # codes 1,7 then 15,0
+    vals = O.decode_e2m1(packed)
+    assert vals.tolist() == [[0.5, 6.0, -6.0, 0.0]]
+
+
+def test_ue4m3_all_bytes_vs_torch_float8():
+    x = np.arange(128, dtype=np.uint8)
+    got = O.decode_ue4m3(x)
+    want = ue4m3_library(x)
+    assert np.isnan(got[0x7F]) and np.isnan(want[0x7F])
+    np.testing.assert_array_equal(got[:0x7F], want[:0x7F])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x38] == 1.0
+    assert np.all(np.diff(got[:0x7F]) > 0)                     # strictly monotone
+
+
+def test_ue4m3_rejects_sign_bit():
+    with pytest.raises(ValueError):
+        O.decode_ue4m3(np.array([0x80], dtype=np.uint8))
+
+
+def test_config_scale_range_is_positive_e4m3_in_quarter_to_four():
+    codes = np.arange(0x28, 0x49, dtype=np.uint8)
+    vals = O.decode_ue4m3(codes)
+    assert len(codes) == 33 and vals[0] == 0.25 and vals[-1] == 4.0
+    allv = ue4m3_library(np.arange(0x7F, dtype=np.uint8))
+    inrange = allv[(allv >= 0.25) & (allv <= 4.0)]
+    np.testing.assert_array_equal(np.sort(inrange), vals)
+
+
+# ---------------------------------------------------------------------------------------
+# 128x4 swizzle
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,k", [(1, 64), (128, 256), (200, 512), (300, 128)])
+def test_swizzle_is_a_bijection_and_matches_permute(rows, k):
+    rp = -(-rows // 128) * 128
+    c = k // 16
+    rr, cc = np.meshgrid(np.arange(rp), np.arange(c), indexing="ij")
+    offs = O.sf_offset(rr, cc, k).ravel()
+    assert sorted(offs.tolist()) == list(range(rp * c))
+    rng = np.random.default_rng(rows + k)
+    logical = rng.integers(0, 127, size=(rows, c), dtype=np.uint8)
+    buf = O.swizzle_scales(logical, k)
+    np.testing.assert_array_equal(buf, swizzle_by_permute(logical, k))
+    np.testing.assert_array_equal(O.unswizzle_scales(buf, rows, k), logical)
+
+
+def test_unswizzle_accepts_larger_buffer_and_rejects_short():
+    logical = np.full((5, 4), 0x38, dtype=np.uint8)
+    buf = O.swizzle_scales(logical, 64)
+    big = np.concatenate([buf, np.full(999, 0x7F, dtype=np.uint8)])
+    np.testing.assert_array_equal(O.unswizzle_scales(big, 5, 64), logical)
+    with pytest.raises(ValueError):
+        O.unswizzle_scales(buf[:-1], 5, 64)
+
+
+# ---------------------------------------------------------------------------------------
+# base product
+# ---------------------------------------------------------------------------------------
+
+def test_single_block_all_byte_pairs():
+    """Every (a byte, b byte) pair in one 16-block: sa*sb*(lo*lo + hi*hi)."""
+    K = 64
+    M = N = 256
+    a = np.zeros((M, K // 2), dtype=np.uint8); a[:, 0] = np.arange(256)
+    b = np.zeros((N, K // 2), dtype=np.uint8); b[:, 0] = np.arange(256)
+    rng = np.random.default_rng(7)
+    sa = rng.integers(0x28, 0x49, size=(M, K // 16), dtype=np.uint8)
+    sb = rng.integers(0x28, 0x49, size=(N, K // 16), dtype=np.uint8)
+    got = O.base_product(a, b, O.swizzle_scales(sa, K), O.swizzle_scales(sb, K), M, N, K)
+    lo = np.array([e2m1_closed_form(i & 15) for i in range(256)])
+    hi = np.array([e2m1_closed_form(i >> 4) for i in range(256)])
+    want = (np.outer(lo, lo) + np.outer(hi, hi)) * np.outer(ue4m3_library(sa[:, 0]),
+                                                            ue4m3_library(sb[:, 0]))
+    np.testing.assert_array_equal(got, want)
+
+
+def test_brute_force_small_random():
+    M, N, K = 3, 5, 128
+    rng = np.random.default_rng(11)
+    a = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    b = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sa = rng.integers(0x01, 0x7F, size=(M, K // 16), dtype=np.uint8)   # full finite range
+    sb = rng.integers(0x01, 0x7F, size=(N, K // 16), dtype=np.uint8)
+    want = brute_base(a, b, sa, sb, M, N, K)
+    got = O.base_product(a, b, swizzle_by_permute(sa, K), swizzle_by_permute(sb, K), M, N, K)
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=0)
+    for m in range(M):
+        for n in range(N):
+            e = O.base_element(a, b, swizzle_by_permute(sa, K), swizzle_by_permute(sb, K),
+                               M, N, K, m, n)
+            assert abs(e - want[m, n]) <= 1e-13 * max(1.0, abs(want[m, n]))
+
+
+def test_all_ones_gives_k():
+    M, N, K = 130, 7, 512
+    a = np.full((M, K // 2), 0x22, dtype=np.uint8)       # both nibbles 1.0
+    b = np.full((N, K // 2), 0x22, dtype=np.uint8)
+    sa = np.full(O.sf_buffer_bytes(M, K), 0x38, dtype=np.uint8)   # 1.0
+    sb = np.full(O.sf_buffer_bytes(N, K), 0x38, dtype=np.uint8)
+    got = O.base_product(a, b, sa, sb, M, N, K)
+    assert np.all(got == K)
+
+
+@pytest.mark.parametrize("k_idx", [0, 1, 15, 16, 17, 63, 64, 65, 127, 191, 255])
+def test_one_hot_lands_on_one_output(k_idx):
+    M, N, K = 40, 140, 256
+    m0, n0 = 37, 133
+    a = np.zeros((M, K // 2), dtype=np.uint8)
+    b = np.zeros((N, K // 2), dtype=np.uint8)
+    a[m0, k_idx // 2] = (0x5 << 4) if k_idx % 2 else 0x5     # 3.0
+    b[n0, k_idx // 2] = (0xB << 4) if k_idx % 2 else 0xB     # -1.5
+    sa_l = np.full((M, K // 16), 0x38, dtype=np.uint8)
+    sb_l = np.full((N, K // 16), 0x38, dtype=np.uint8)
+    sa_l[m0, k_idx // 16] = 0x40          # 2.0
+    sb_l[n0, k_idx // 16] = 0x29          # 0.28125
+    got = O.base_product(a, b, swizzle_by_permute(sa_l, K), swizzle_by_permute(sb_l, K),
+                         M, N, K)
+    want = np.zeros((M, N)); want[m0, n0] = 3.0 * -1.5 * 2.0 * 0.28125
+    np.testing.assert_array_equal(got, want)
+
+
+def test_golden_hand_computed_case():
+    with open(os.path.join(GOLDEN, "hand_case.json")) as f:
+        g = json.load(f)
+    M, N, K, r = g["M"], g["N"], g["K"], g["r"]
+    a = np.array(g["a"], dtype=np.uint8).reshape(M, K // 2)
+    b = np.array(g["b"], dtype=np.uint8).reshape(N, K // 2)
+    sa = O.swizzle_scales(np.array(g["a_sf_logical"], dtype=np.uint8).reshape(M, K // 16), K)
+    sb = O.swizzle_scales(np.array(g["b_sf_logical"], dtype=np.uint8).reshape(N, K // 16), K)
+    d = np.array(g["d_bits"], dtype=np.uint16)
+    lb = np.array(g["lora_b_bits"], dtype=np.uint16)
+    bias = np.array(g["bias_bits"], dtype=np.uint16)
+    y = O.mm_raw(a, b, sa, sb, g["alpha"], d, lb, g["lora_scale"], bias, M, N, K, r)
+    np.testing.assert_array_equal(y.ravel(), np.array(g["expected_y"]))
+    np.testing.assert_array_equal(O.round_output(y).ravel(),
+                                  np.array(g["expected_out_bits"], dtype=np.uint16))
+
+
+# ---------------------------------------------------------------------------------------
+# rounding
+# ---------------------------------------------------------------------------------------
+
+def test_f64_to_bf16_matches_torch_on_float32_values():
+    rng = np.random.default_rng(3)
+    bits = rng.integers(0, 2 ** 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    x32 = bits.view(np.float32)
+    x32 = x32[~np.isnan(x32)]
+    got = O.f64_to_bf16_rne(x32.astype(np.float64))
+    want = torch.from_numpy(x32.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(got, want)
+    got32 = O.f32_to_bf16_rne(x32)
+    np.testing.assert_array_equal(got32, want)
+
+
+def test_f64_to_bf16_single_rounding_cases():
+    one = 1.0
+    cases = [
+        (one + 2.0 ** -8, 0x3F80),                    # tie -> even (down)
+        (one + 2.0 ** -8 + 2.0 ** -40, 0x3F81),       # just above the tie: up (f32 route says down)
+        (one + 3 * 2.0 ** -8, 0x3F82),                # tie -> even (up)
+        (-(one + 2.0 ** -8 + 2.0 ** -40), 0xBF81),
+        ((2 - 2.0 ** -8) * 2.0 ** 127, 0x7F80),       # tie at the top -> even = infinity
+        ((2 - 2.0 ** -8 - 2.0 ** -30) * 2.0 ** 127, 0x7F7F),
+        (2.0 ** -133, 0x0001),                        # smallest subnormal
+        (2.0 ** -134, 0x0000),                        # tie -> even (zero)
+        (1.5 * 2.0 ** -134, 0x0001),
+        (2.0 ** -126, 0x0080),                        # smallest normal
+        (0.0, 0x0000),
+        (-0.0, 0x8000),
+        (float("inf"), 0x7F80),
+        (float("-inf"), 0xFF80),
+        (1e300, 0x7F80),
+    ]
+    ys = np.array([c[0] for c in cases])
+    got = O.f64_to_bf16_rne(ys)
+    assert [int(v) for v in got] == [c[1] for c in cases]
+    assert int(O.f64_to_bf16_rne(np.array([float("nan")]))[0]) == 0x7FC0
+
+
+# ---------------------------------------------------------------------------------------
+# fold
+# ---------------------------------------------------------------------------------------
+
+FOLD_PAIRS = [(0.25, 2.0 ** -10), (2.0, 2.0 ** -9), (0.5, 3.0), (1.7, -0.013), (0.0, 2.0 ** -9),
+              (-0.0, 1.0), (3.999, 1e-30), (1e-30, 3.0), (7.0, 1e-38)]
+
+
+@pytest.mark.parametrize("s,alpha", FOLD_PAIRS)
+def test_fold_matches_torch_mul_exhaustive(s, alpha):
+    lb_bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ratio, got = O.fold(lb_bits, s, alpha)
+    st = torch.tensor([s], dtype=torch.float32)
+    at = torch.tensor([alpha], dtype=torch.float32)
+    rt = (st / at[0])
+    assert np.float32(rt.item()) == ratio or (np.isnan(ratio) and math.isnan(rt.item()))
+    lb = torch.from_numpy(lb_bits.view(np.int16).copy()).view(torch.bfloat16)
+    want = (lb * rt[0]).view(torch.int16).numpy().view(np.uint16)
+    gotf = (got.astype(np.uint32) << 16).view(np.float32)
+    wantf = (want.astype(np.uint32) << 16).view(np.float32)
+    nan_g, nan_w = np.isnan(gotf), np.isnan(wantf)
+    np.testing.assert_array_equal(nan_g, nan_w)
+    np.testing.assert_array_equal(got[~nan_g], want[~nan_w])
+    assert np.all(got[nan_g] == 0x7FC0)
+
+
+def test_fold_exact_when_ratio_is_power_of_two():
+    rng = np.random.default_rng(5)
+    lb = (torch.from_numpy(rng.standard_normal(4096).astype(np.float32)) * 0.02).to(torch.bfloat16)
+    bits = lb.view(torch.int16).numpy().view(np.uint16)
+    ratio, folded = O.fold(bits, 0.25, 2.0 ** -10)
+    assert ratio == np.float32(256.0)
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(folded), O.bf16_bits_to_f64(bits) * 256.0)
+
+
+def test_eager_checks():
+    with pytest.raises(ValueError):
+        O.eager_prepare_check(1.0, 0.0)
+    with pytest.raises(ValueError):
+        O.eager_prepare_check(1.0, -0.0)
+    with pytest.raises(ValueError):
+        O.eager_prepare_check(3e38, 1e-10)       # ratio overflows
+    with pytest.raises(ValueError):
+        O.eager_prepare_check(float("nan"), 1.0)
+    O.eager_prepare_check(0.0, 1.0)               # the zero adapter is allowed
+
+
+# ---------------------------------------------------------------------------------------
+# epilogue algebra and invariants
+# ---------------------------------------------------------------------------------------
+
+def _small_problem(seed, M=33, N=70, K=256, r=16, bias=True):
+    from workloads import make_problem
+    p = make_problem(M, N, K, r, seed, alpha=2.0 ** -6, lora_scale=1.5, bias=bias)
+    npy = dict(a=p.a.numpy(), b=p.b.numpy(), a_sf=p.a_sf.numpy(), b_sf=p.b_sf.numpy(),
+               d=p.d.view(torch.int16).numpy().view(np.uint16),
+               lb=p.lora_b.view(torch.int16).numpy().view(np.uint16),
+               bias=None if p.bias is None else p.bias.view(torch.int16).numpy().view(np.uint16))
+    return p, npy
+
+
+def test_zero_adapter_is_bitwise_adapter_off_even_with_nonfinite_d():
+    p, x = _small_problem(21)
+    d = x["d"].copy(); d[0, 0] = 0x7F80; d[1, 3] = 0x7FC1       # inf, NaN
+    off = O.mm_off(x["a"], x["b"], x["a_sf"], x["b_sf"], p.alpha, x["bias"], p.M, p.N, p.K)
+    for s in (0.0, -0.0, None):
+        raw = O.mm_raw(x["a"], x["b"], x["a_sf"], x["b_sf"], p.alpha, d, x["lb"], s, x["bias"],
+                       p.M, p.N, p.K, p.r)
+        np.testing.assert_array_equal(raw.view(np.uint64), off.view(np.uint64))
+    prep = O.mm_prepared(x["a"], x["b"], x["a_sf"], x["b_sf"], p.alpha, d, x["lb"], 0.0,
+                         x["bias"], p.M, p.N, p.K, p.r)
+    np.testing.assert_array_equal(prep.view(np.uint64), off.view(np.uint64))
+
+
+def test_raw_minus_off_is_the_lora_term_closed_form():
+    """alpha = 0 isolates s * (d @ lora_b^T) + bias, checked by an explicit loop."""
+    p, x = _small_problem(22, M=5, N=9, r=24)
+    y = O.mm_raw(x["a"], x["b"], x["a_sf"], x["b_sf"], 0.0, x["d"], x["lb"], 1.5, x["bias"],
+                 p.M, p.N, p.K, p.r)
+    d = p.d.double().numpy(); lb = p.lora_b.double().numpy(); bias = p.bias.double().numpy()
+    for m in range(p.M):
+        for n in range(p.N):
+            want = 1.5 * sum(d[m, j] * lb[n, j] for j in range(p.r)) + bias[n]
+            assert abs(y[m, n] - want) <= 1e-14 * max(1.0, abs(want))
+
+
+def test_raw_vs_prepared_agree_within_fold_rounding():
+    p, x = _small_problem(23, M=64, N=96, r=32)
+    for s, alpha in [(1.5, 2.0 ** -6), (0.3, 0.0071)]:
+        ratio, bf = O.fold(x["lb"], s, alpha)
+        y_raw = O.mm_raw(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], x["lb"], s,
+                         x["bias"], p.M, p.N, p.K, p.r)
+        y_prep = O.mm_prepared(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], bf, ratio,
+                               x["bias"], p.M, p.N, p.K, p.r)
+        d = np.abs(O.bf16_bits_to_f64(x["d"])); lb = np.abs(O.bf16_bits_to_f64(x["lb"]))
+        bound = abs(s) * (d @ lb.T) * (2.0 ** -9 + 2.0 ** -22) + 1e-12 * np.abs(y_raw)
+        assert np.all(np.abs(y_raw - y_prep) <= bound)
+        assert np.any(y_raw != y_prep) or s == 1.5   # the fold does change something
+
+
+def test_raw_vs_prepared_equal_when_fold_is_exact():
+    p, x = _small_problem(24, M=32, N=48, r=64, bias=False)
+    s, alpha = 0.25, 2.0 ** -10          # ratio 256, exact
+    ratio, bf = O.fold(x["lb"], s, alpha)
+    y_raw = O.mm_raw(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], x["lb"], s, None,
+                     p.M, p.N, p.K, p.r)
+    y_prep = O.mm_prepared(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], bf, ratio, None,
+                           p.M, p.N, p.K, p.r)
+    np.testing.assert_allclose(y_prep, y_raw, rtol=1e-15, atol=1e-300)
+
+
+def test_measures():
+    y = np.array([1.0, -2.0, 4.0])
+    assert O.sqnr_db(y, y) == float("inf")
+    assert abs(O.sqnr_db(y, y + np.array([0.0, 0.0, 0.21])) - 10 * np.log10(21 / 0.0441)) < 1e-9
+    np.testing.assert_array_equal(O.tolerance(y), 2.0 ** -7 * np.abs(y) + 2.0 ** -10 * 4.0)

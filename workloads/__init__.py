@@ -1,0 +1,109 @@
+"""Seeded synthetic inputs shared by the tests, ``bench.py`` and ``smoke()``.
+
+This module draws random bytes and numbers and nothing else: it holds none of the
+operation's arithmetic (no decoding, no swizzle arithmetic, no products), so the CPU
+oracle and the CUDA path can both take their inputs from it without sharing code.
+
+Value distributions follow the workloads stated for the operation
+(flashinfer.gemm.mm_nvfp4_lora: E2M1 codes uniform over the 16 codes, UE4M3 block
+scales uniform over the positive E4M3 values in [0.25, 4], d ~ N(0, 1), lora_b ~
+N(0, 0.02), bias ~ N(0, 0.1)), drawn with ``torch.Generator`` on the CPU in a fixed
+order: a, b, a_sf, b_sf, d, lora_b, bias.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+#: positive E4M3 bytes 0x28 (0.25) .. 0x48 (4.0): 33 codes, all finite and normal
+SF_LO = 0x28
+SF_HI = 0x48
+
+
+def sf_bytes(rows: int, k: int) -> int:
+    """Bytes of a scale buffer whose rows are padded to a multiple of 128."""
+    return -(-rows // 128) * 128 * (k // 16)
+
+
+@dataclasses.dataclass
+class Problem:
+    """One GEMM problem's host tensors (CPU, contiguous)."""
+    M: int
+    N: int
+    K: int
+    r: int
+    a: torch.Tensor          # uint8 [M, K/2]
+    b: torch.Tensor          # uint8 [N, K/2]
+    a_sf: torch.Tensor       # uint8 [padded(M) * K/16], swizzled layout, drawn bytewise
+    b_sf: torch.Tensor       # uint8 [padded(N) * K/16]
+    alpha: float
+    lora_scale: Optional[float]
+    d: Optional[torch.Tensor]        # bf16 [M, r]
+    lora_b: Optional[torch.Tensor]   # bf16 [N, r]
+    bias: Optional[torch.Tensor]     # bf16 [N]
+
+
+def make_problem(M: int, N: int, K: int, r: int, seed: int, *, alpha: float,
+                 lora_scale: Optional[float], bias: bool, d_std: float = 1.0,
+                 lb_std: float = 0.02, bias_std: float = 0.1,
+                 codes: str = "uniform") -> Problem:
+    """Draw one problem.  Every byte of the padded scale buffers is drawn (padding rows
+    included), so no knowledge of the swizzle is needed here."""
+    g = torch.Generator().manual_seed(seed)
+    if codes == "uniform":
+        a = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.uint8)
+        b = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
+    elif codes == "zero":
+        a = torch.zeros((M, K // 2), dtype=torch.uint8)
+        b = torch.zeros((N, K // 2), dtype=torch.uint8)
+    else:
+        raise ValueError(codes)
+    a_sf = torch.randint(SF_LO, SF_HI + 1, (sf_bytes(M, K),), generator=g, dtype=torch.uint8)
+    b_sf = torch.randint(SF_LO, SF_HI + 1, (sf_bytes(N, K),), generator=g, dtype=torch.uint8)
+    d = (torch.randn(M, r, generator=g) * d_std).to(torch.bfloat16)
+    lora_b = (torch.randn(N, r, generator=g) * lb_std).to(torch.bfloat16)
+    bias_t = (torch.randn(N, generator=g) * bias_std).to(torch.bfloat16) if bias else None
+    return Problem(M, N, K, r, a, b, a_sf, b_sf, alpha, lora_scale, d, lora_b, bias_t)
+
+
+def make_adapters(N: int, r: int, count: int, seed: int, lb_std: float = 0.02):
+    """``count`` adapters: lora_b ~ N(0, lb_std) bf16 [N, r], lora_scale ~ U[0.1, 4]."""
+    g = torch.Generator().manual_seed(seed)
+    out = []
+    for _ in range(count):
+        lb = (torch.randn(N, r, generator=g) * lb_std).to(torch.bfloat16)
+        s = float(torch.empty(1).uniform_(0.1, 4.0, generator=g).item())
+        out.append((lb, s))
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# The workloads (shapes, paths and scalars).  "cfg0" is the small parity case; "cfg1" is
+# the decode shape the throughput metric is quoted on at M <= 16; "cfg2"/"cfg3" are the
+# prefill and large MLP-up shapes; "cfg4" is the adapter-switch sweep.
+# --------------------------------------------------------------------------------------
+
+CONFIGS = {
+    "cfg0": dict(M=128, N=256, K=256, r=16, path="raw", alpha=2.0 ** -6, lora_scale=2.0,
+                 bias=False, seed=0),
+    "cfg1": dict(M=16, N=4096, K=4096, r=64, path="raw", alpha=2.0 ** -9, lora_scale=0.5,
+                 bias=True, seed=1),
+    "cfg2": dict(M=4096, N=4096, K=4096, r=16, path="raw", alpha=2.0 ** -9, lora_scale=2.0,
+                 bias=True, seed=2),
+    "cfg3": dict(M=8192, N=28672, K=8192, r=64, path="prepared", alpha=2.0 ** -10,
+                 lora_scale=0.25, bias=False, seed=3),
+}
+
+#: adapter-switch sweep: N=14336, K=4096, M x r grid, 8 adapters, alpha 2**-9
+CFG4 = dict(N=14336, K=4096, Ms=(1, 32, 256, 2048), rs=(8, 128), adapters=8,
+            alpha=2.0 ** -9, seed=4)
+
+
+def config_problem(name: str, **over) -> Problem:
+    c = dict(CONFIGS[name])
+    c.update(over)
+    return make_problem(c["M"], c["N"], c["K"], c["r"], c["seed"], alpha=c["alpha"],
+                        lora_scale=c["lora_scale"], bias=c["bias"])
