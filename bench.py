@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Throughput of the NVFP4 + LoRA GEMM on B200, against its roofline, with the CPU oracle
+timed beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg1] [--impl ours|reference]
+
+One step = one call of the workload's path (raw: nvfp4lora_mm; prepared: refold + GEMM for
+the adapter-switch workloads).  The default workload is the decode shape M=16, N=4096,
+K=4096, r=64 (raw path with bias), whose metric is HBM GB/s; compute-bound workloads report
+TFLOPS.  Weights are rotated through enough copies (>= 3x the L2 size in total) that every
+step reads them from HBM; steps are CUDA-graph replays timed with CUDA events on the
+launching stream.  N > 1 (torchrun): every rank runs its own independent problem (weak
+scaling, no collective on the data path); the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "NVFP4+LoRA GEMM TFLOPS and % of FP4 tensor peak (HBM GB/s % at M<=16)"
+PROFILES = os.path.join(ROOT, "profiles")
+
+# workload name -> (config key or explicit dict, path, default steps)
+WORKLOADS = {
+    "cfg0": dict(src="cfg0", steps=2000),
+    "cfg1": dict(src="cfg1", steps=20000),
+    "cfg2": dict(src="cfg2", steps=2000),
+    "cfg3": dict(src="cfg3", steps=100),
+}
+
+
+def describe(name):
+    from workloads import CONFIGS
+    c = dict(CONFIGS[WORKLOADS[name]["src"]])
+    return c
+
+
+def algorithmic(c):
+    """Algorithmic bytes and flops of one call (padded scale rows and operand re-reads are
+    implementation overhead and excluded)."""
+    M, N, K, r = c["M"], c["N"], c["K"], c["r"]
+    nbytes = (M * K // 2 + N * K // 2 + M * K // 16 + N * K // 16 + M * r * 2 + N * r * 2
+              + (N * 2 if c["bias"] else 0) + M * N * 2 + 4 + 4)
+    return nbytes, 2 * M * N * K, 2 * M * N * r
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            j = json.load(f)
+        return j, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "nvfp4_block_scaled_mm_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(PROFILES, f"gemm_{workload}_traffic.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha") != source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period_s=0.01):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, device):
+    import nvfp4_block_scaled_mm_b200 as L
+    from workloads import make_problem
+
+    c = describe(args.workload)
+    M, N, K, r = c["M"], c["N"], c["K"], c["r"]
+    p = make_problem(M, N, K, r, c["seed"] + 1000 * rank, alpha=c["alpha"], lora_scale=c["lora_scale"],
+                     bias=c["bias"])
+    nbytes, flops, lora_flops = algorithmic(c)
+    in_bytes = sum(t.numel() * t.element_size() for t in (p.a, p.b, p.a_sf, p.b_sf, p.d, p.lora_b)) + \
+        (p.bias.numel() * 2 if p.bias is not None else 0)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(1, math.ceil(3 * l2 / in_bytes))
+
+    def dev(t):
+        return None if t is None else t.to(device)
+
+    sets = []
+    for _ in range(copies):
+        sets.append(dict(a=dev(p.a), b=dev(p.b), a_sf=dev(p.a_sf), b_sf=dev(p.b_sf), d=dev(p.d),
+                         lora_b=dev(p.lora_b), bias=dev(p.bias)))
+    alpha = torch.tensor([c["alpha"]], dtype=torch.float32, device=device)
+    s = torch.tensor([c["lora_scale"]], dtype=torch.float32, device=device)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    prepared = c["path"] == "prepared"
+    adapters = []
+    if prepared:
+        for st in sets:
+            adapters.append(L.prepare_nvfp4_lora_adapter(st["lora_b"], s, alpha))
+
+    def step(i):
+        st = sets[i % copies]
+        if prepared:
+            adp = adapters[i % copies]
+            L.prepare_nvfp4_lora_adapter(st["lora_b"], s, alpha, out=adp)
+            L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, st["d"], lora_adapter=adp,
+                            bias=st["bias"], out=out)
+        else:
+            L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, st["d"], st["lora_b"], s,
+                            bias=st["bias"], out=out)
+
+    K_steps = args.steps if args.steps is not None else WORKLOADS[args.workload]["steps"]
+    W = args.warmup
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(max(W, 3)):      # eager warm-up (also sets kernel attributes)
+            step(i)
+        L.nvfp4lora_device_status(stream)
+        g_warm = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_warm, stream=stream):
+            for i in range(max(W, 3)):
+                step(i)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(K_steps):
+                step(i)
+    launches_per_step = 2 if prepared else 1
+
+    torch.cuda.synchronize(device)
+    g_warm.replay()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            g.replay()
+            end.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    L.nvfp4lora_device_status(stream)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / K_steps
+
+    # end to end through the public API with host buffers: per step, the activation-side
+    # inputs (a, a_sf, d) go host -> device and the output comes back device -> host.
+    e2e = run_e2e(L, p, sets[0], alpha, s, out, c, device, stream, min(K_steps, 2000), prepared,
+                  adapters[0] if prepared else None)
+
+    return dict(c=c, ms=ms, ms_step=ms_step, K=K_steps, W=max(W, 3), nbytes=nbytes, flops=flops,
+                lora_flops=lora_flops, copies=copies, clocks=clk.summary(), e2e=e2e,
+                launches=K_steps * launches_per_step, in_bytes=in_bytes, l2=l2, p=p)
+
+
+def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
+    a_h = p.a.pin_memory()
+    a_sf_h = p.a_sf.pin_memory()
+    d_h = p.d.pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    a_d, a_sf_d, d_d = torch.empty_like(st["a"]), torch.empty_like(st["a_sf"]), torch.empty_like(st["d"])
+    h2d = a_h.numel() + a_sf_h.numel() + d_h.numel() * 2
+    d2h = out.numel() * 2
+
+    def one():
+        a_d.copy_(a_h, non_blocking=True)
+        a_sf_d.copy_(a_sf_h, non_blocking=True)
+        d_d.copy_(d_h, non_blocking=True)
+        if prepared:
+            L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, lora_adapter=adp, bias=st["bias"], out=out)
+        else:
+            L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, st["lora_b"], s, bias=st["bias"], out=out)
+        out_h.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    return dict(ms_step=ms, steps=steps, h2d=h2d, d2h=d2h)
+
+
+# ---------------------------------------------------------------------------------------
+# the oracle as the CPU baseline / reference arm
+# ---------------------------------------------------------------------------------------
+
+def oracle_sample(p, c, ncols):
+    """Oracle on all M rows x the first `ncols` output columns of the workload; returns the
+    fraction of the workload's outputs this covers."""
+    import oracle as O
+    a = p.a.numpy(); b = p.b.numpy(); a_sf = p.a_sf.numpy(); b_sf = p.b_sf.numpy()
+    dbits = p.d.view(torch.int16).numpy().view(np.uint16)
+    lbits = p.lora_b.view(torch.int16).numpy().view(np.uint16)
+    rows = np.arange(c["M"])
+    cols = np.arange(ncols)
+    base = O.base_product_rows_cols(a, b, a_sf, b_sf, c["K"], rows, cols)
+    dd = O.bf16_bits_to_f64(dbits.reshape(c["M"], c["r"]))
+    if c["path"] == "prepared":
+        ratio, bf = O.fold(lbits[:ncols], c["lora_scale"], c["alpha"])
+        lb = O.bf16_bits_to_f64(bf.reshape(ncols, c["r"]))
+        y = c["alpha"] * (base + dd @ lb.T)
+    else:
+        lb = O.bf16_bits_to_f64(lbits.reshape(c["N"], c["r"])[:ncols])
+        y = c["alpha"] * base + c["lora_scale"] * (dd @ lb.T)
+        if p.bias is not None:
+            y = y + O.bf16_bits_to_f64(p.bias.view(torch.int16).numpy().view(np.uint16)[:ncols])[None, :]
+    O.round_output(y)
+    return ncols / c["N"]
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def calibrate_cols(p, c, budget_s):
+    ncols = min(c["N"], 64)
+    t0 = time.perf_counter()
+    oracle_sample(p, c, ncols)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    want = int(ncols * budget_s / dt)
+    return max(8, min(c["N"], want))
+
+
+def cpu_baseline(p, c, nbytes, flops, budget_s=12.0):
+    """Time the oracle on a bounded sample of the workload for about `budget_s` seconds."""
+    ncols = calibrate_cols(p, c, budget_s / 3)
+    t0 = time.perf_counter()
+    reps = 0
+    frac = 0.0
+    while True:
+        frac += oracle_sample(p, c, ncols)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    value, unit = metric_value(c, nbytes * frac / reps, flops * frac / reps, dt / reps * 1e3)
+    return dict(value=value, unit=unit, cores=oracle_threads(), kind="oracle",
+                sample=f"{reps} x oracle on all {c['M']} rows x the first {ncols} of {c['N']} output columns "
+                       f"({frac / reps:.4f} of the workload each), {dt:.1f} s")
+
+
+def metric_value(c, nbytes, flops, ms):
+    if c["M"] <= 16:
+        return nbytes / (ms * 1e-3) / 1e9, "GB/s"
+    return flops / (ms * 1e-3) / 1e12, "TFLOPS"
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the oracle, as it stands, timed on the host cores on the same
+    workload, one bounded sample per step."""
+    from workloads import make_problem
+    if rank != 0:
+        return 0
+    c = describe(args.workload)
+    p = make_problem(c["M"], c["N"], c["K"], c["r"], c["seed"], alpha=c["alpha"],
+                     lora_scale=c["lora_scale"], bias=c["bias"])
+    nbytes, flops, _ = algorithmic(c)
+    K_steps = args.steps if args.steps is not None else 20
+    W = args.warmup
+    per_step_budget = max(0.01, 120.0 / (K_steps + W))
+    ncols = calibrate_cols(p, c, per_step_budget)
+    for _ in range(W):
+        oracle_sample(p, c, ncols)
+    t0 = time.perf_counter()
+    frac = 0.0
+    for _ in range(K_steps):
+        frac += oracle_sample(p, c, ncols)
+    dt = time.perf_counter() - t0
+    ms_step = dt / K_steps * 1e3
+    value, unit = metric_value(c, nbytes * frac / K_steps, flops * frac / K_steps, ms_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
+        "steps": K_steps, "warmup": W, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(args, c),
+        "cpu_baseline": {"value": value, "unit": unit, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"each step: oracle on all {c['M']} rows x the first {ncols} of {c['N']} "
+                                   f"output columns ({ncols / c['N']:.4f} of the workload)"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(args, c):
+    return {"workload": f"{args.workload}: M={c['M']} N={c['N']} K={c['K']} r={c['r']} {c['path']} path"
+                        f"{' + bias' if c['bias'] else ''}",
+            "M": c["M"], "N": c["N"], "K": c["K"], "r": c["r"], "path": c["path"],
+            "alpha": c["alpha"], "lora_scale": c["lora_scale"], "bias": c["bias"],
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
+            "l2_defeat": "weights and activations rotate through copies totalling >= 3x L2",
+            "timing": "CUDA graph of K back-to-back calls, CUDA events on the launching stream"}
+
+
+# ---------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg1")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=device,
+                                             timeout=datetime.timedelta(seconds=120))
+    res = run_ours(args, rank, world, device)
+    c = res["c"]
+    value, unit = metric_value(c, res["nbytes"], res["flops"], res["ms_step"])
+    peaks, peak_src = measured_peaks()
+    if unit == "GB/s":
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
+                "peak_source": f"hbm_gbs of {peak_src}"}
+    else:
+        # FP4 dense peak = measured bf16 (sustained, long step) x nominal fp4/bf16 ratio (9 / 2.25)
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 4.0
+        roof = {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                "peak_source": f"bf16_tflops_sustained x 4 (nominal fp4/bf16) of {peak_src}"}
+    traffic = recorded_traffic(args.workload)
+    roof["traffic"] = traffic
+    roof["algorithmic_bytes_per_launch"] = res["nbytes"]
+    e2e = res["e2e"]
+    e2e_val, e2e_unit = metric_value(c, res["nbytes"], res["flops"], e2e["ms_step"] * 1.0)
+    line = {
+        "metric": METRIC, "value": value * world, "unit": unit, "n_gpus": world, "steps": res["K"],
+        "warmup": res["W"], "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3 -> fp32) + bf16 LoRA", "data": "synthetic",
+        "config": config_block(args, c), "roofline": roof, "clocks": res["clocks"],
+        "e2e": {"value": e2e_val * world, "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"],
+                "note": "per step: a, a_sf, d host->device (pinned), call, out device->host; weights resident"},
+        "gpu_launches": res["launches"],
+        "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
+        "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(res["p"], c, res["nbytes"], res["flops"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

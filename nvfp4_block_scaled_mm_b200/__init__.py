@@ -1,0 +1,313 @@
+"""NVFP4 block-scaled GEMM with a fused BF16 LoRA correction on B200 (sm_100a).
+
+Thin ctypes binding over the C ABI in ``include/nvfp4lora.h`` (``libnvfp4lora.so``, built
+in-tree by :mod:`nvfp4_block_scaled_mm_b200.build`).  It only marshals arguments: every
+step of the operation runs in the library's CUDA kernels.  PyTorch supplies device
+memory, the current stream and the tensors' version counters (used for the stale-adapter
+check).  There is no CPU fallback: the library is loaded on first use, and a missing
+library raises ``RuntimeError`` there.
+
+Two layers:
+
+* ``nvfp4lora_mm``, ``nvfp4lora_prepare``, ``nvfp4lora_refold``,
+  ``nvfp4lora_mm_prepared`` -- one-to-one with the C entry points (torch tensors in, the
+  status mapped to exceptions);
+* ``mm_nvfp4_lora``, ``prepare_nvfp4_lora_adapter``, ``PreparedNvFp4LoraAdapter``,
+  ``StaleAdapterError`` -- the API of flashinfer.gemm.mm_nvfp4_lora and
+  flashinfer.gemm.prepare_nvfp4_lora_adapter (signatures, Parameters, Returns, Notes).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .build import LIB_PATH
+
+__all__ = [
+    "StaleAdapterError", "PreparedNvFp4LoraAdapter", "mm_nvfp4_lora", "prepare_nvfp4_lora_adapter",
+    "nvfp4lora_mm", "nvfp4lora_prepare", "nvfp4lora_refold", "nvfp4lora_mm_prepared",
+    "nvfp4lora_device_status", "library_path", "version",
+]
+
+OK, INVALID_ARG, STALE, ALPHA_ZERO, UNSUPPORTED_ARCH, DEVICE_TIMEOUT, CUDA_ERR = range(7)
+
+
+class StaleAdapterError(RuntimeError):
+    """A prepared adapter's alpha, lora_b or lora_scale changed since its last (re)fold."""
+
+
+class DeviceTimeoutError(RuntimeError):
+    """A kernel's bounded wait ran out (reported by :func:`nvfp4lora_device_status`)."""
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m nvfp4_block_scaled_mm_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, U64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int32
+    lib.nvfp4lora_mm.argtypes = [P, P, P, I64, P, I64, P, P, P, P, I64, P, P, I64, I64, I64, P]
+    lib.nvfp4lora_mm.restype = ctypes.c_int
+    lib.nvfp4lora_prepare.argtypes = [P, P, P, I64, I64, P, P, U64, P, P]
+    lib.nvfp4lora_prepare.restype = ctypes.c_int
+    lib.nvfp4lora_refold.argtypes = [P, P, P, P, I64, I64, U64, P]
+    lib.nvfp4lora_refold.restype = ctypes.c_int
+    lib.nvfp4lora_mm_prepared.argtypes = [P, P, P, I64, P, I64, P, P, P, P, P, U64, P, P, I64, I64, I64, P]
+    lib.nvfp4lora_mm_prepared.restype = ctypes.c_int
+    lib.nvfp4lora_device_status.argtypes = [P]
+    lib.nvfp4lora_device_status.restype = ctypes.c_int
+    lib.nvfp4lora_last_error.argtypes = []
+    lib.nvfp4lora_last_error.restype = ctypes.c_char_p
+    lib.nvfp4lora_version.argtypes = []
+    lib.nvfp4lora_version.restype = ctypes.c_char_p
+    del I32
+    return lib
+
+
+class _LazyLib:
+    """Loads libnvfp4lora.so on first attribute access (raises if it was never built)."""
+
+    _handle = None
+
+    def __getattr__(self, name):
+        if _LazyLib._handle is None:
+            _LazyLib._handle = _load()
+        return getattr(_LazyLib._handle, name)
+
+
+_lib = _LazyLib()
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library():
+    """Load the CUDA library now (it is otherwise loaded on first use)."""
+    _lib.nvfp4lora_version  # noqa: B018
+    return LIB_PATH
+
+
+def version() -> str:
+    return _lib.nvfp4lora_version().decode()
+
+
+class _Adapter(ctypes.Structure):
+    _fields_ = [("b_folded", ctypes.c_void_p), ("ratio", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("lora_b", ctypes.c_void_p), ("lora_scale", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("r", ctypes.c_int64), ("src_version", ctypes.c_uint64), ("device", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+def _check(status: int) -> None:
+    if status == OK:
+        return
+    msg = _lib.nvfp4lora_last_error().decode()
+    if status in (INVALID_ARG, ALPHA_ZERO):
+        raise ValueError(msg)
+    if status == STALE:
+        raise StaleAdapterError(msg)
+    if status == DEVICE_TIMEOUT:
+        raise DeviceTimeoutError(msg)
+    raise RuntimeError(msg)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _version_token(lora_b: torch.Tensor, lora_scale: torch.Tensor) -> int:
+    return ((lora_b._version & 0xFFFFFFFF) << 32) | (lora_scale._version & 0xFFFFFFFF)
+
+
+# --------------------------------------------------------------------------------------
+# one-to-one C ABI wrappers
+# --------------------------------------------------------------------------------------
+
+def nvfp4lora_mm(a, b, a_sf, b_sf, alpha, d, lora_b, lora_scale, r, bias, out, M, N, K, stream=None):
+    _check(_lib.nvfp4lora_mm(_ptr(a), _ptr(b), _ptr(a_sf), a_sf.numel(), _ptr(b_sf), b_sf.numel(),
+                             _ptr(alpha), _ptr(d), _ptr(lora_b), _ptr(lora_scale), int(r), _ptr(bias),
+                             _ptr(out), int(M), int(N), int(K), _stream(stream)))
+    return out
+
+
+def nvfp4lora_prepare(lora_b, lora_scale, alpha, N, r, b_folded, ratio, src_version, stream=None):
+    adp = _Adapter()
+    _check(_lib.nvfp4lora_prepare(_ptr(lora_b), _ptr(lora_scale), _ptr(alpha), int(N), int(r),
+                                  _ptr(b_folded), _ptr(ratio), int(src_version), ctypes.byref(adp),
+                                  _stream(stream)))
+    return adp
+
+
+def nvfp4lora_refold(adp, lora_b, lora_scale, alpha, N, r, src_version, stream=None):
+    _check(_lib.nvfp4lora_refold(ctypes.byref(adp), _ptr(lora_b), _ptr(lora_scale), _ptr(alpha),
+                                 int(N), int(r), int(src_version), _stream(stream)))
+    return adp
+
+
+def nvfp4lora_mm_prepared(a, b, a_sf, b_sf, alpha, d, adp, cur_lora_b, cur_lora_scale, cur_version,
+                          bias, out, M, N, K, stream=None):
+    _check(_lib.nvfp4lora_mm_prepared(_ptr(a), _ptr(b), _ptr(a_sf), a_sf.numel(), _ptr(b_sf),
+                                      b_sf.numel(), _ptr(alpha), _ptr(d), ctypes.byref(adp),
+                                      _ptr(cur_lora_b), _ptr(cur_lora_scale), int(cur_version),
+                                      _ptr(bias), _ptr(out), int(M), int(N), int(K), _stream(stream)))
+    return out
+
+
+def nvfp4lora_device_status(stream=None) -> None:
+    """Synchronise the stream and raise DeviceTimeoutError if a kernel's wait ran out."""
+    _check(_lib.nvfp4lora_device_status(_stream(stream)))
+
+
+# --------------------------------------------------------------------------------------
+# the pages' API
+# --------------------------------------------------------------------------------------
+
+def _need(t, name, dtype, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+
+
+class PreparedNvFp4LoraAdapter:
+    """A folded adapter (prepare_nvfp4_lora_adapter, Returns): ``b_folded`` bf16 [N, r], the
+    device ``ratio`` scalar, the alpha tensor it belongs to, and the pins of its sources."""
+
+    def __init__(self, c_adapter: _Adapter, b_folded, ratio, alpha, lora_b, lora_scale):
+        self._c = c_adapter
+        self.b_folded = b_folded
+        self.ratio = ratio
+        self.alpha = alpha
+        self.lora_b = lora_b
+        self.lora_scale = lora_scale
+
+    @property
+    def N(self) -> int:
+        return int(self._c.N)
+
+    @property
+    def r(self) -> int:
+        return int(self._c.r)
+
+
+def _check_fold_inputs(lora_b, lora_scale, alpha):
+    _need(lora_b, "lora_b", torch.bfloat16, 2)
+    _need(lora_scale, "lora_scale", torch.float32)
+    _need(alpha, "alpha", torch.float32)
+    if lora_scale.numel() != 1:
+        raise ValueError("lora_scale must be a one-element fp32 tensor")
+    if alpha.numel() < 1:
+        raise ValueError("alpha must hold at least one element")
+
+
+def prepare_nvfp4_lora_adapter(lora_b: torch.Tensor, lora_scale: torch.Tensor, alpha: torch.Tensor, *,
+                               out: Optional[PreparedNvFp4LoraAdapter] = None) -> PreparedNvFp4LoraAdapter:
+    """Fold ``b_folded = bf16(lora_b * (lora_scale / alpha[0]))``.
+
+    ``out=None``: the eager form (one host read of (lora_scale, alpha); alpha == 0 or a
+    non-finite ratio raises ValueError).  ``out=adapter``: in-place refold on the device,
+    no host read, graph-capturable; alpha must be the adapter's own alpha tensor.
+    """
+    _check_fold_inputs(lora_b, lora_scale, alpha)
+    N, r = lora_b.shape
+    stream = torch.cuda.current_stream(lora_b.device)
+    if out is None:
+        with torch.cuda.device(lora_b.device):
+            b_folded = torch.empty_like(lora_b)
+            ratio = torch.empty(1, dtype=torch.float32, device=lora_b.device)
+            c = nvfp4lora_prepare(lora_b, lora_scale, alpha, N, r, b_folded, ratio,
+                                  _version_token(lora_b, lora_scale), stream)
+        return PreparedNvFp4LoraAdapter(c, b_folded, ratio, alpha, lora_b, lora_scale)
+    if not isinstance(out, PreparedNvFp4LoraAdapter):
+        raise ValueError("out must be a PreparedNvFp4LoraAdapter")
+    with torch.cuda.device(lora_b.device):
+        nvfp4lora_refold(out._c, lora_b, lora_scale, alpha, N, r, _version_token(lora_b, lora_scale), stream)
+    out.lora_b = lora_b
+    out.lora_scale = lora_scale
+    return out
+
+
+def mm_nvfp4_lora(a: torch.Tensor, b: torch.Tensor, a_sf: torch.Tensor, b_sf: torch.Tensor,
+                  alpha: torch.Tensor, d: Optional[torch.Tensor] = None,
+                  lora_b: Optional[torch.Tensor] = None, lora_scale: Optional[torch.Tensor] = None, *,
+                  lora_adapter: Optional[PreparedNvFp4LoraAdapter] = None,
+                  bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  out_dtype: torch.dtype = torch.bfloat16, backend: str = "cake",
+                  enable_pdl: Optional[bool] = None) -> torch.Tensor:
+    """``out = alpha * (dequant(a) @ dequant(b)^T) + lora_scale * (d @ lora_b^T) [+ bias]``.
+
+    Raw path: ``d``, ``lora_b``, ``lora_scale``; ``lora_scale=None`` is the adapter-off
+    call even if d / lora_b are given.  Prepared path: ``lora_adapter=`` plus ``d``.
+    """
+    if out_dtype != torch.bfloat16:
+        raise ValueError("out_dtype: only torch.bfloat16 is supported")
+    if backend not in ("cake", "auto"):
+        raise ValueError("backend must be 'cake' or 'auto'")
+    if enable_pdl not in (None, True):
+        raise ValueError("enable_pdl must be None or True")
+    if lora_adapter is not None and (lora_b is not None or lora_scale is not None):
+        raise ValueError("pass either the raw adapter (lora_b, lora_scale) or lora_adapter, not both")
+    _need(a, "a", torch.uint8, 2)
+    _need(b, "b", torch.uint8, 2)
+    _need(a_sf, "a_sf", torch.uint8)
+    _need(b_sf, "b_sf", torch.uint8)
+    _need(alpha, "alpha", torch.float32)
+    M, K = a.shape[0], a.shape[1] * 2
+    N = b.shape[0]
+    if b.shape[1] * 2 != K:
+        raise ValueError(f"a is [M, K/2] = {tuple(a.shape)} but b is {tuple(b.shape)}: K differs")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 1)
+        if bias.shape[0] != N:
+            raise ValueError(f"bias must be [N] = [{N}]")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    else:
+        _need(out, "out", torch.bfloat16, 2)
+        if tuple(out.shape) != (M, N):
+            raise ValueError(f"out must be [M, N] = [{M}, {N}]")
+    stream = torch.cuda.current_stream(a.device)
+    with torch.cuda.device(a.device):
+        if lora_adapter is not None:
+            if d is None:
+                raise ValueError("the prepared path still requires d")
+            _need(d, "d", torch.bfloat16, 2)
+            if tuple(d.shape) != (M, lora_adapter.r):
+                raise ValueError(f"d must be [M, r] = [{M}, {lora_adapter.r}]")
+            src = lora_adapter
+            nvfp4lora_mm_prepared(a, b, a_sf, b_sf, alpha, d, src._c, src.lora_b, src.lora_scale,
+                                  _version_token(src.lora_b, src.lora_scale), bias, out, M, N, K, stream)
+            return out
+        if lora_scale is None:
+            nvfp4lora_mm(a, b, a_sf, b_sf, alpha, None, None, None, 0, bias, out, M, N, K, stream)
+            return out
+        _need(lora_scale, "lora_scale", torch.float32)
+        if lora_scale.numel() != 1:
+            raise ValueError("lora_scale must be a one-element fp32 tensor")
+        if d is None or lora_b is None:
+            raise ValueError("the raw path needs d and lora_b with lora_scale")
+        _need(d, "d", torch.bfloat16, 2)
+        _need(lora_b, "lora_b", torch.bfloat16, 2)
+        r = d.shape[1]
+        if d.shape[0] != M or tuple(lora_b.shape) != (N, r):
+            raise ValueError(f"d must be [M, r] and lora_b [N, r]; got {tuple(d.shape)}, {tuple(lora_b.shape)}")
+        nvfp4lora_mm(a, b, a_sf, b_sf, alpha, d, lora_b, lora_scale, r, bias, out, M, N, K, stream)
+        return out

@@ -1,0 +1,422 @@
+// C ABI of the NVFP4 + LoRA GEMM library (declared in include/nvfp4lora.h).
+//
+// Host side: argument rules (flashinfer.gemm.mm_nvfp4_lora, Notes: Shape rules; Parameters),
+// adapter pins and stale checks (Parameters: lora_adapter; Notes: CUDA graphs), the eager
+// prepare's single host read and checks (prepare_nvfp4_lora_adapter, Parameters: alpha,
+// Returns), TMA descriptor encoding, and kernel launch.  Every rule is checked before any
+// CUDA call, so a rejected call enqueues nothing.  This is the library's only translation
+// unit: it includes the kernels and the device error word they set.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/nvfp4lora.h"
+#include "fold.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace nvfp4lora {
+namespace {
+
+thread_local std::string t_last_error;
+
+nvfp4lora_status fail(nvfp4lora_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return st;
+}
+
+nvfp4lora_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(NVFP4LORA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------------------------------
+// device facts, cached per device
+// ---------------------------------------------------------------------------------------
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool init = false;
+    bool supported = false;
+    int sms = 0;
+    int major = 0, minor = 0;
+    bool gemm_attr_set[3] = {false, false, false};
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+nvfp4lora_status device_info(int* dev_out, DeviceInfo** info_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(NVFP4LORA_ERR_CUDA, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.init) {
+        if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        d.supported = (d.major == 10 && d.minor == 0);
+        d.init = true;
+    }
+    if (!d.supported)
+        return fail(NVFP4LORA_ERR_UNSUPPORTED_ARCH,
+                    "device %d is sm_%d%d; this library runs on sm_100 (B200) only", dev, d.major, d.minor);
+    *dev_out = dev;
+    *info_out = &d;
+    return NVFP4LORA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// TMA descriptors
+// ---------------------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+cudaError_t g_encode_err = cudaSuccess;
+
+nvfp4lora_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        g_encode_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (g_encode_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (g_encode == nullptr)
+        return fail(NVFP4LORA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)",
+                    cudaGetErrorString(g_encode_err));
+    *out = g_encode;
+    return NVFP4LORA_OK;
+}
+
+// 2-D row-major tensor [rows, cols] of `esize`-byte elements, read in boxes of
+// box_cols x box_rows with the 128-byte swizzle; out-of-range elements read as zero.
+nvfp4lora_status encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int esize,
+                           uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    nvfp4lora_status st = get_encoder(&enc);
+    if (st != NVFP4LORA_OK) return st;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)esize};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4LORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return NVFP4LORA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// argument rules
+// ---------------------------------------------------------------------------------------
+
+constexpr int64_t kMaxDim = (int64_t)1 << 30;   // keeps every tile coordinate in int32
+constexpr int64_t kMaxK = (int64_t)1 << 20;
+
+nvfp4lora_status check_rank(int64_t r) {
+    if (r < 8 || r > 128 || r % 8 != 0)
+        return fail(NVFP4LORA_ERR_INVALID_ARG,
+                    "LoRA rank r = %lld: r must be a multiple of 8 in [8, 128]", (long long)r);
+    return NVFP4LORA_OK;
+}
+
+nvfp4lora_status check_base(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, int64_t a_sf_bytes,
+                            const uint8_t* b_sf, int64_t b_sf_bytes, const float* alpha,
+                            const uint16_t* bias, const uint16_t* out, int64_t M, int64_t N, int64_t K) {
+    if (M < 1) return fail(NVFP4LORA_ERR_INVALID_ARG, "M = %lld: M >= 1 is required", (long long)M);
+    if (N < 1) return fail(NVFP4LORA_ERR_INVALID_ARG, "N = %lld: N >= 1 is required", (long long)N);
+    if (K < 256 || K % 256 != 0)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "K = %lld: K must be a positive multiple of 256", (long long)K);
+    if (M > kMaxDim || N > kMaxDim || K > kMaxK)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "M, N <= 2^30 and K <= 2^20 are required");
+    if (!a || !b || !a_sf || !b_sf || !alpha || !out)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "a, b, a_sf, b_sf, alpha and out must be non-null");
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) || !aligned(out, 16))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "a, b, a_sf, b_sf and out must be 16-byte aligned");
+    if (!aligned(alpha, 4)) return fail(NVFP4LORA_ERR_INVALID_ARG, "alpha must be 4-byte aligned");
+    if (bias && !aligned(bias, 2)) return fail(NVFP4LORA_ERR_INVALID_ARG, "bias must be 2-byte aligned");
+    const int64_t need_a = (M + 127) / 128 * 128 * (K / 16);
+    const int64_t need_b = (N + 127) / 128 * 128 * (K / 16);
+    if (a_sf_bytes < need_a)
+        return fail(NVFP4LORA_ERR_INVALID_ARG,
+                    "a_sf has %lld bytes; the 128x4 layout with rows padded to 128 needs %lld",
+                    (long long)a_sf_bytes, (long long)need_a);
+    if (b_sf_bytes < need_b)
+        return fail(NVFP4LORA_ERR_INVALID_ARG,
+                    "b_sf has %lld bytes; the 128x4 layout with rows padded to 128 needs %lld",
+                    (long long)b_sf_bytes, (long long)need_b);
+    return NVFP4LORA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// GEMM launch
+// ---------------------------------------------------------------------------------------
+
+constexpr int kBN = 128;
+constexpr int kStages = 6;
+
+template <Mode MODE>
+nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                             const float* alpha, const float* scale, const uint16_t* d,
+                             const uint16_t* lb, int64_t r, const uint16_t* bias, uint16_t* out,
+                             int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    int dev;
+    DeviceInfo* info;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+
+    auto kernel = nvfp4_gemm_kernel<kBN, kStages, MODE>;
+    constexpr int smem = GemmSmem<kBN, kStages>::DYN_BYTES;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!info->gemm_attr_set[(int)MODE]) {
+            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+            info->gemm_attr_set[(int)MODE] = true;
+        }
+    }
+
+    CUtensorMap tm_a, tm_b, tm_d, tm_lb;
+    std::memset(&tm_d, 0, sizeof(tm_d));
+    std::memset(&tm_lb, 0, sizeof(tm_lb));
+    if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) != NVFP4LORA_OK) return st;
+    if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, kBN)) != NVFP4LORA_OK) return st;
+    if (MODE != Mode::Off) {
+        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, kBN)) != NVFP4LORA_OK) return st;
+    }
+
+    GemmArgs args;
+    args.a_sf = a_sf;
+    args.b_sf = b_sf;
+    args.alpha = alpha;
+    args.scale = scale;
+    args.bias = bias;
+    args.out = out;
+    args.M = (int)M;
+    args.N = (int)N;
+    args.K = (int)K;
+    args.r = (int)r;
+    args.m_tiles = (int)((M + 127) / 128);
+    args.n_tiles = (int)((N + kBN - 1) / kBN);
+    const int64_t tiles = (int64_t)args.m_tiles * args.n_tiles;
+    if (tiles > INT32_MAX) return fail(NVFP4LORA_ERR_INVALID_ARG, "too many output tiles (M x N too large)");
+    args.num_tiles = (int)tiles;
+    args.k_stages = (int)(K / 256);
+    args.sf_atoms_k = (int)(K / 64);
+    args.sf_row_blocks_b = (int)((N + 127) / 128);
+
+    const int grid = (int)std::min<int64_t>(tiles, info->sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, args);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+    return NVFP4LORA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// fold launch
+// ---------------------------------------------------------------------------------------
+
+nvfp4lora_status launch_fold(const uint16_t* lora_b, const float* lora_scale, const float* alpha,
+                             uint16_t* b_folded, float* ratio, int64_t N, int64_t r, cudaStream_t stream) {
+    int dev;
+    DeviceInfo* info;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+    const int64_t groups = N * r / 8;
+    const int64_t want = (groups + kFoldThreads - 1) / kFoldThreads;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)info->sms * 8));
+    fold_kernel<<<grid, kFoldThreads, 0, stream>>>(lora_b, lora_scale, alpha, b_folded, ratio, groups);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "fold launch");
+    return NVFP4LORA_OK;
+}
+
+nvfp4lora_status check_fold_args(const uint16_t* lora_b, const float* lora_scale, const float* alpha,
+                                  int64_t N, int64_t r, const uint16_t* b_folded, const float* ratio) {
+    if (N < 1) return fail(NVFP4LORA_ERR_INVALID_ARG, "N = %lld: N >= 1 is required", (long long)N);
+    if (N > kMaxDim) return fail(NVFP4LORA_ERR_INVALID_ARG, "N <= 2^30 is required");
+    nvfp4lora_status st = check_rank(r);
+    if (st != NVFP4LORA_OK) return st;
+    if (!lora_b || !lora_scale || !alpha || !b_folded || !ratio)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_b, lora_scale, alpha, b_folded and ratio must be non-null");
+    if (!aligned(lora_b, 16) || !aligned(b_folded, 16))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_b and b_folded must be 16-byte aligned");
+    if (!aligned(lora_scale, 4) || !aligned(alpha, 4) || !aligned(ratio, 4))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_scale, alpha and ratio must be 4-byte aligned");
+    if (ratio == lora_scale || ratio == alpha)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "ratio must not alias lora_scale or alpha");
+    return NVFP4LORA_OK;
+}
+
+}  // namespace
+}  // namespace nvfp4lora
+
+using namespace nvfp4lora;
+
+extern "C" {
+
+nvfp4lora_status nvfp4lora_mm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, int64_t a_sf_bytes,
+                              const uint8_t* b_sf, int64_t b_sf_bytes, const float* alpha,
+                              const uint16_t* d, const uint16_t* lora_b, const float* lora_scale, int64_t r,
+                              const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                              nvfp4lora_stream stream) {
+    t_last_error.clear();
+    nvfp4lora_status st = check_base(a, b, a_sf, a_sf_bytes, b_sf, b_sf_bytes, alpha, bias, out, M, N, K);
+    if (st != NVFP4LORA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (lora_scale == nullptr)
+        return launch_gemm<Mode::Off>(a, b, a_sf, b_sf, alpha, nullptr, nullptr, nullptr, 0, bias, out, M, N, K, s);
+    if ((st = check_rank(r)) != NVFP4LORA_OK) return st;
+    if (!d || !lora_b) return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_scale given: d and lora_b must be non-null");
+    if (!aligned(d, 16) || !aligned(lora_b, 16))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "d and lora_b must be 16-byte aligned");
+    if (!aligned(lora_scale, 4)) return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_scale must be 4-byte aligned");
+    return launch_gemm<Mode::Raw>(a, b, a_sf, b_sf, alpha, lora_scale, d, lora_b, r, bias, out, M, N, K, s);
+}
+
+nvfp4lora_status nvfp4lora_prepare(const uint16_t* lora_b, const float* lora_scale, const float* alpha,
+                                   int64_t N, int64_t r, uint16_t* b_folded, float* ratio,
+                                   uint64_t src_version, nvfp4lora_adapter* adapter_out,
+                                   nvfp4lora_stream stream) {
+    t_last_error.clear();
+    if (!adapter_out) return fail(NVFP4LORA_ERR_INVALID_ARG, "adapter_out must be non-null");
+    nvfp4lora_status st = check_fold_args(lora_b, lora_scale, alpha, N, r, b_folded, ratio);
+    if (st != NVFP4LORA_OK) return st;
+    int dev;
+    DeviceInfo* info;
+    if ((st = device_info(&dev, &info)) != NVFP4LORA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // The single host read of the adapter switch: (lora_scale, alpha).
+    float host[2] = {0.0f, 0.0f};
+    cudaError_t e = cudaMemcpyAsync(&host[0], lora_scale, sizeof(float), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&host[1], alpha, sizeof(float), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading lora_scale and alpha");
+    if (host[1] == 0.0f)
+        return fail(NVFP4LORA_ERR_ALPHA_ZERO, "alpha == 0: lora_scale / alpha is undefined "
+                                              "(the alpha == 0 LoRA-only call is the raw path)");
+    volatile float q = host[0] / host[1];
+    if (!std::isfinite((float)q))
+        return fail(NVFP4LORA_ERR_ALPHA_ZERO, "lora_scale / alpha = %g is not finite", (double)q);
+    if ((st = launch_fold(lora_b, lora_scale, alpha, b_folded, ratio, N, r, s)) != NVFP4LORA_OK) return st;
+    adapter_out->b_folded = b_folded;
+    adapter_out->ratio = ratio;
+    adapter_out->alpha = alpha;
+    adapter_out->lora_b = lora_b;
+    adapter_out->lora_scale = lora_scale;
+    adapter_out->N = N;
+    adapter_out->r = r;
+    adapter_out->src_version = src_version;
+    adapter_out->device = dev;
+    adapter_out->reserved = 0;
+    return NVFP4LORA_OK;
+}
+
+nvfp4lora_status nvfp4lora_refold(nvfp4lora_adapter* adapter, const uint16_t* lora_b, const float* lora_scale,
+                                  const float* alpha, int64_t N, int64_t r, uint64_t src_version,
+                                  nvfp4lora_stream stream) {
+    t_last_error.clear();
+    if (!adapter) return fail(NVFP4LORA_ERR_INVALID_ARG, "adapter must be non-null");
+    nvfp4lora_status st = check_fold_args(lora_b, lora_scale, alpha, N, r, adapter->b_folded, adapter->ratio);
+    if (st != NVFP4LORA_OK) return st;
+    if (alpha != adapter->alpha)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "alpha must be the adapter's own alpha tensor");
+    if (N != adapter->N || r != adapter->r)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_b must keep the adapter's [N, r] = [%lld, %lld]",
+                    (long long)adapter->N, (long long)adapter->r);
+    int dev;
+    DeviceInfo* info;
+    if ((st = device_info(&dev, &info)) != NVFP4LORA_OK) return st;
+    if (dev != adapter->device)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_b must stay on the adapter's device %d", adapter->device);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = launch_fold(lora_b, lora_scale, alpha, adapter->b_folded, adapter->ratio, N, r, s)) != NVFP4LORA_OK)
+        return st;
+    adapter->lora_b = lora_b;
+    adapter->lora_scale = lora_scale;
+    adapter->src_version = src_version;
+    return NVFP4LORA_OK;
+}
+
+nvfp4lora_status nvfp4lora_mm_prepared(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, int64_t a_sf_bytes,
+                                       const uint8_t* b_sf, int64_t b_sf_bytes, const float* alpha,
+                                       const uint16_t* d, const nvfp4lora_adapter* adapter,
+                                       const uint16_t* cur_lora_b, const float* cur_lora_scale,
+                                       uint64_t cur_src_version, const uint16_t* bias, uint16_t* out,
+                                       int64_t M, int64_t N, int64_t K, nvfp4lora_stream stream) {
+    t_last_error.clear();
+    nvfp4lora_status st = check_base(a, b, a_sf, a_sf_bytes, b_sf, b_sf_bytes, alpha, bias, out, M, N, K);
+    if (st != NVFP4LORA_OK) return st;
+    if (!adapter) return fail(NVFP4LORA_ERR_INVALID_ARG, "adapter must be non-null");
+    if (!adapter->b_folded || !adapter->ratio)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "adapter has no b_folded / ratio buffers");
+    if (adapter->N != N)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "adapter has N = %lld, the call N = %lld",
+                    (long long)adapter->N, (long long)N);
+    if ((st = check_rank(adapter->r)) != NVFP4LORA_OK) return st;
+    if (!d) return fail(NVFP4LORA_ERR_INVALID_ARG, "the prepared path still requires d");
+    if (!aligned(d, 16) || !aligned(adapter->b_folded, 16))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "d and b_folded must be 16-byte aligned");
+    if (alpha != adapter->alpha)
+        return fail(NVFP4LORA_ERR_STALE_ADAPTER,
+                    "the adapter was prepared for another alpha tensor; re-prepare when alpha changes");
+    if (cur_lora_b != adapter->lora_b || cur_lora_scale != adapter->lora_scale)
+        return fail(NVFP4LORA_ERR_STALE_ADAPTER, "the adapter's lora_b / lora_scale moved since the prepare");
+    if (cur_src_version != adapter->src_version)
+        return fail(NVFP4LORA_ERR_STALE_ADAPTER, "the adapter's lora_b / lora_scale were written since the prepare");
+    int dev;
+    DeviceInfo* info;
+    if ((st = device_info(&dev, &info)) != NVFP4LORA_OK) return st;
+    if (dev != adapter->device)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "the adapter lives on device %d, the call runs on %d",
+                    adapter->device, dev);
+    return launch_gemm<Mode::Prepared>(a, b, a_sf, b_sf, alpha, adapter->ratio, d, adapter->b_folded,
+                                       adapter->r, bias, out, M, N, K, reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream) {
+    t_last_error.clear();
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (word != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+        return fail(NVFP4LORA_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (pipeline stalled)");
+    }
+    return NVFP4LORA_OK;
+}
+
+const char* nvfp4lora_last_error(void) { return t_last_error.c_str(); }
+
+const char* nvfp4lora_version(void) { return "nvfp4lora 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -210,6 +210,22 @@ def base_element(a, b, a_sf, b_sf, M: int, N: int, K: int, m: int, n: int) -> fl
     return total
 
 
+def dequant_rows(codes, sf_buf, K: int, rows) -> np.ndarray:
+    """``dequant`` of selected rows only (for sampled checks at full sizes)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    codes = np.asarray(codes, dtype=np.uint8).reshape(-1, K // 2)
+    vals = decode_e2m1(codes[rows])
+    cols = np.arange(K // SF_VEC)
+    offs = sf_offset(rows[:, None], cols[None, :], K)
+    scales = decode_ue4m3(np.asarray(sf_buf, dtype=np.uint8).reshape(-1)[offs])
+    return vals * np.repeat(scales, SF_VEC, axis=1)
+
+
+def base_product_rows_cols(a, b, a_sf, b_sf, K: int, rows, cols) -> np.ndarray:
+    """The base product restricted to ``rows`` x ``cols`` (same definition, fewer outputs)."""
+    return dequant_rows(a, a_sf, K, rows) @ dequant_rows(b, b_sf, K, cols).T
+
+
 def lora_term(d_bits, lb_bits, M: int, N: int, r: int) -> np.ndarray:
     """``d @ lora_b^T`` in float64 (bf16 x bf16 products are exact in float64)."""
     d = bf16_bits_to_f64(np.asarray(d_bits).reshape(M, r))
@@ -273,7 +289,7 @@ def round_output(y: np.ndarray) -> np.ndarray:
 
 def fold_ratio(lora_scale: float, alpha: float) -> np.float32:
     """``div.rn.f32(fp32(lora_scale), fp32(alpha[0]))``: one IEEE binary32 division."""
-    with np.errstate(divide="ignore", invalid="ignore"):
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
         return np.float32(lora_scale) / np.float32(alpha)
 
 

@@ -1,0 +1,108 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the header
+declares, and rejects rule violations before touching CUDA (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4lora.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_block_scaled_mm_b200.build import build
+    path = build(quiet=True)
+    return ctypes.CDLL(path)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NVFP4LORA_API\s+[\w\s\*]+?\b(nvfp4lora_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("nvfp4lora_mm", "nvfp4lora_prepare", "nvfp4lora_refold", "nvfp4lora_mm_prepared",
+                 "nvfp4lora_device_status", "nvfp4lora_last_error", "nvfp4lora_version"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_binding_exposes_the_same_names():
+    import nvfp4_block_scaled_mm_b200 as L
+    for name in declared_symbols():
+        if name in ("nvfp4lora_last_error", "nvfp4lora_version"):
+            continue
+        assert callable(getattr(L, name)), name
+
+
+P = ctypes.c_void_p
+I64 = ctypes.c_int64
+
+
+def _mm(lib, **kw):
+    f = lib.nvfp4lora_mm
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, I64, P, I64, P, P, P, P, I64, P, P, I64, I64, I64, P]
+    lib.nvfp4lora_last_error.restype = ctypes.c_char_p
+    args = dict(a=0x10000, b=0x20000, a_sf=0x30000, a_sf_bytes=1 << 30, b_sf=0x40000, b_sf_bytes=1 << 30,
+                alpha=0x50000, d=0x60000, lora_b=0x70000, lora_scale=0x80000, r=16, bias=None,
+                out=0x90000, M=128, N=256, K=256)
+    args.update(kw)
+    st = f(args["a"], args["b"], args["a_sf"], args["a_sf_bytes"], args["b_sf"], args["b_sf_bytes"],
+           args["alpha"], args["d"], args["lora_b"], args["lora_scale"], args["r"], args["bias"], args["out"],
+           args["M"], args["N"], args["K"], None)
+    return st, lib.nvfp4lora_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,needle", [
+    (dict(M=0), "M >= 1"),
+    (dict(N=0), "N >= 1"),
+    (dict(K=300), "multiple of 256"),
+    (dict(K=0), "multiple of 256"),
+    (dict(r=12), "multiple of 8"),
+    (dict(r=136), "multiple of 8"),
+    (dict(r=0), "multiple of 8"),
+    (dict(a=0x10004), "16-byte aligned"),
+    (dict(out=0x90002), "16-byte aligned"),
+    (dict(alpha=None), "non-null"),
+    (dict(d=None), "d and lora_b"),
+    (dict(a_sf_bytes=128 * 16 - 1), "a_sf has"),
+    (dict(M=129, a_sf_bytes=128 * 16), "a_sf has"),
+    (dict(N=257, b_sf_bytes=256 * 16), "b_sf has"),
+    (dict(M=1 << 31), "2^30"),
+])
+def test_rule_violations_are_rejected_before_cuda(lib, kw, needle):
+    st, msg = _mm(lib, **kw)
+    assert st == 1, (st, msg)
+    assert needle in msg, msg
+
+
+def test_adapter_off_ignores_rank(lib):
+    """lora_scale = NULL is the adapter-off call: a bad r is not a violation there.  (The
+    call then proceeds to CUDA, which fails without a GPU with a CUDA status, not 1.)"""
+    st, msg = _mm(lib, lora_scale=None, r=3, d=None, lora_b=None)
+    assert st != 1, msg
+
+
+def test_prepare_rules(lib):
+    f = lib.nvfp4lora_prepare
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, I64, I64, P, P, ctypes.c_uint64, P, P]
+    buf = ctypes.create_string_buffer(128)
+    assert f(0x1000, 0x2000, 0x3000, 16, 12, 0x4000, 0x5000, 0, buf, None) == 1
+    assert f(0x1000, 0x2000, 0x3000, 0, 16, 0x4000, 0x5000, 0, buf, None) == 1
+    assert f(0x1000, 0x2000, 0x3000, 16, 16, 0x4000, 0x2000, 0, buf, None) == 1   # ratio aliases lora_scale
+    assert f(0x1000, 0x2000, 0x3000, 16, 16, 0x4000, 0x5000, 0, None, None) == 1
+
+
+def test_version_string(lib):
+    lib.nvfp4lora_version.restype = ctypes.c_char_p
+    assert b"sm_100a" in lib.nvfp4lora_version()
