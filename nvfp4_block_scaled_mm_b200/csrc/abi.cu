@@ -17,11 +17,13 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <set>
 #include <string>
 
 #include "../../include/nvfp4lora.h"
 #include "fold.cuh"
 #include "gemm.cuh"
+#include "gemm_decode.cuh"
 #include "ptx.cuh"
 
 namespace nvfp4lora {
@@ -56,7 +58,7 @@ struct DeviceInfo {
     bool supported = false;
     int sms = 0;
     int major = 0, minor = 0;
-    bool gemm_attr_set[3] = {false, false, false};
+    std::set<const void*> smem_attr_set;   // kernels whose dynamic shared memory limit is raised
 };
 
 std::mutex g_mu;
@@ -82,6 +84,17 @@ nvfp4lora_status device_info(int* dev_out, DeviceInfo** info_out) {
                     "device %d is sm_%d%d; this library runs on sm_100 (B200) only", dev, d.major, d.minor);
     *dev_out = dev;
     *info_out = &d;
+    return NVFP4LORA_OK;
+}
+
+template <typename Kernel>
+nvfp4lora_status ensure_smem_attr(DeviceInfo* info, Kernel kernel, int smem) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    const void* key = reinterpret_cast<const void*>(kernel);
+    if (info->smem_attr_set.count(key)) return NVFP4LORA_OK;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    info->smem_attr_set.insert(key);
     return NVFP4LORA_OK;
 }
 
@@ -180,21 +193,14 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
                              const float* alpha, const float* scale, const uint16_t* d,
                              const uint16_t* lb, int64_t r, const uint16_t* bias, uint16_t* out,
                              int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
-    int dev;
-    DeviceInfo* info;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
     nvfp4lora_status st = device_info(&dev, &info);
     if (st != NVFP4LORA_OK) return st;
 
     auto kernel = nvfp4_gemm_kernel<kBN, kStages, MODE>;
     constexpr int smem = GemmSmem<kBN, kStages>::DYN_BYTES;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (!info->gemm_attr_set[(int)MODE]) {
-            cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-            info->gemm_attr_set[(int)MODE] = true;
-        }
-    }
+    if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
     CUtensorMap tm_a, tm_b, tm_d, tm_lb;
     std::memset(&tm_d, 0, sizeof(tm_d));
@@ -238,13 +244,108 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
 }
 
 // ---------------------------------------------------------------------------------------
+// decode launch (M <= kDecodeMaxM): swapped operands, split-K over a cluster
+// ---------------------------------------------------------------------------------------
+
+constexpr int kDecodeMaxM = 32;
+constexpr int kDecodeStages = 8;
+
+// Largest cluster split S in {8, 4, 2, 1} that keeps n_tiles * S CTAs within one wave and
+// divides the K stages.
+int decode_splits(int n_tiles, int k_stages, int sms) {
+    for (int s = 8; s > 1; s >>= 1)
+        if (k_stages % s == 0 && (int64_t)n_tiles * s <= sms) return s;
+    return 1;
+}
+
+template <int MT, Mode MODE>
+nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint8_t* b, const uint8_t* a_sf,
+                                  const uint8_t* b_sf, const float* alpha, const float* scale, const uint16_t* d,
+                                  const uint16_t* lb, int64_t r, const uint16_t* bias, uint16_t* out,
+                                  int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    nvfp4lora_status st;
+    auto kernel = nvfp4_decode_kernel<MT, kDecodeStages, MODE>;
+    constexpr int smem = DecodeSmem<MT, kDecodeStages>::DYN_BYTES;
+    if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
+
+    CUtensorMap tm_a, tm_b, tm_d, tm_lb;
+    std::memset(&tm_d, 0, sizeof(tm_d));
+    std::memset(&tm_lb, 0, sizeof(tm_lb));
+    if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, MT)) != NVFP4LORA_OK) return st;
+    if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) != NVFP4LORA_OK) return st;
+    if (MODE != Mode::Off) {
+        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, MT)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, 128)) != NVFP4LORA_OK) return st;
+    }
+    DecodeArgs args;
+    args.a_sf = a_sf;
+    args.b_sf = b_sf;
+    args.alpha = alpha;
+    args.scale = scale;
+    args.bias = bias;
+    args.out = out;
+    args.M = (int)M;
+    args.N = (int)N;
+    args.K = (int)K;
+    args.r = (int)r;
+    args.n_tiles = (int)((N + 127) / 128);
+    const int k_stages = (int)(K / 256);
+    args.splits = decode_splits(args.n_tiles, k_stages, info->sms);
+    args.stages_per_split = k_stages / args.splits;
+    args.sf_atoms_k = (int)(K / 64);
+    args.sf_row_blocks_b = (int)((N + 127) / 128);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(args.n_tiles, args.splits);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    if (args.splits > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = args.splits;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, args);
+    if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
+    return NVFP4LORA_OK;
+}
+
+template <Mode MODE>
+nvfp4lora_status launch_decode(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                               const float* alpha, const float* scale, const uint16_t* d, const uint16_t* lb,
+                               int64_t r, const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                               cudaStream_t stream) {
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+    if (M <= 16)
+        return launch_decode_mt<16, MODE>(info, a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
+    return launch_decode_mt<32, MODE>(info, a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
+}
+
+// Chooses the decode kernel for M <= 32 and the tiled kernel otherwise.
+template <Mode MODE>
+nvfp4lora_status launch(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                        const float* alpha, const float* scale, const uint16_t* d, const uint16_t* lb, int64_t r,
+                        const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    if (M <= kDecodeMaxM)
+        return launch_decode<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
+    return launch_gemm<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
+}
+
+// ---------------------------------------------------------------------------------------
 // fold launch
 // ---------------------------------------------------------------------------------------
 
 nvfp4lora_status launch_fold(const uint16_t* lora_b, const float* lora_scale, const float* alpha,
                              uint16_t* b_folded, float* ratio, int64_t N, int64_t r, cudaStream_t stream) {
-    int dev;
-    DeviceInfo* info;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
     nvfp4lora_status st = device_info(&dev, &info);
     if (st != NVFP4LORA_OK) return st;
     const int64_t groups = N * r / 8;
@@ -290,13 +391,13 @@ nvfp4lora_status nvfp4lora_mm(const uint8_t* a, const uint8_t* b, const uint8_t*
     if (st != NVFP4LORA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (lora_scale == nullptr)
-        return launch_gemm<Mode::Off>(a, b, a_sf, b_sf, alpha, nullptr, nullptr, nullptr, 0, bias, out, M, N, K, s);
+        return launch<Mode::Off>(a, b, a_sf, b_sf, alpha, nullptr, nullptr, nullptr, 0, bias, out, M, N, K, s);
     if ((st = check_rank(r)) != NVFP4LORA_OK) return st;
     if (!d || !lora_b) return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_scale given: d and lora_b must be non-null");
     if (!aligned(d, 16) || !aligned(lora_b, 16))
         return fail(NVFP4LORA_ERR_INVALID_ARG, "d and lora_b must be 16-byte aligned");
     if (!aligned(lora_scale, 4)) return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_scale must be 4-byte aligned");
-    return launch_gemm<Mode::Raw>(a, b, a_sf, b_sf, alpha, lora_scale, d, lora_b, r, bias, out, M, N, K, s);
+    return launch<Mode::Raw>(a, b, a_sf, b_sf, alpha, lora_scale, d, lora_b, r, bias, out, M, N, K, s);
 }
 
 nvfp4lora_status nvfp4lora_prepare(const uint16_t* lora_b, const float* lora_scale, const float* alpha,
@@ -307,8 +408,8 @@ nvfp4lora_status nvfp4lora_prepare(const uint16_t* lora_b, const float* lora_sca
     if (!adapter_out) return fail(NVFP4LORA_ERR_INVALID_ARG, "adapter_out must be non-null");
     nvfp4lora_status st = check_fold_args(lora_b, lora_scale, alpha, N, r, b_folded, ratio);
     if (st != NVFP4LORA_OK) return st;
-    int dev;
-    DeviceInfo* info;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
     if ((st = device_info(&dev, &info)) != NVFP4LORA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // The single host read of the adapter switch: (lora_scale, alpha).
@@ -349,8 +450,8 @@ nvfp4lora_status nvfp4lora_refold(nvfp4lora_adapter* adapter, const uint16_t* lo
     if (N != adapter->N || r != adapter->r)
         return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_b must keep the adapter's [N, r] = [%lld, %lld]",
                     (long long)adapter->N, (long long)adapter->r);
-    int dev;
-    DeviceInfo* info;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
     if ((st = device_info(&dev, &info)) != NVFP4LORA_OK) return st;
     if (dev != adapter->device)
         return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_b must stay on the adapter's device %d", adapter->device);
@@ -389,13 +490,13 @@ nvfp4lora_status nvfp4lora_mm_prepared(const uint8_t* a, const uint8_t* b, const
         return fail(NVFP4LORA_ERR_STALE_ADAPTER, "the adapter's lora_b / lora_scale moved since the prepare");
     if (cur_src_version != adapter->src_version)
         return fail(NVFP4LORA_ERR_STALE_ADAPTER, "the adapter's lora_b / lora_scale were written since the prepare");
-    int dev;
-    DeviceInfo* info;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
     if ((st = device_info(&dev, &info)) != NVFP4LORA_OK) return st;
     if (dev != adapter->device)
         return fail(NVFP4LORA_ERR_INVALID_ARG, "the adapter lives on device %d, the call runs on %d",
                     adapter->device, dev);
-    return launch_gemm<Mode::Prepared>(a, b, a_sf, b_sf, alpha, adapter->ratio, d, adapter->b_folded,
+    return launch<Mode::Prepared>(a, b, a_sf, b_sf, alpha, adapter->ratio, d, adapter->b_folded,
                                        adapter->r, bias, out, M, N, K, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -56,25 +56,35 @@ def finish():
 # ---------------------------------------------------------------------------------------
 
 @pytest.mark.parametrize("s,alpha", [(0.25, 2.0 ** -10), (2.0, 2.0 ** -9), (1.7, -0.013), (0.0, 0.5),
-                                     (3.999, 1e-30), (7.0, 1e-38)])
+                                     (3.999, 1e-30), (7.0, 1e-38), (1.0, 0.0), (0.0, 0.0)])
 def test_fold_bitwise_all_bf16_patterns(s, alpha):
+    """Eager fold (finite ratio) and in-place refold (any ratio) are bitwise the oracle's fold
+    over all 65536 bf16 patterns; a non-finite ratio is refused by the eager form only."""
     lb_bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     lb = torch.from_numpy(lb_bits.view(np.int16).copy()).view(torch.bfloat16).reshape(512, 128).cuda()
     st = torch.tensor([s], dtype=torch.float32, device="cuda")
     at = torch.tensor([alpha], dtype=torch.float32, device="cuda")
-    adp = L.prepare_nvfp4_lora_adapter(lb, st, at)
-    finish()
     ratio, want = O.fold(lb_bits, s, alpha)
-    got_ratio = adp.ratio.cpu().numpy()[0]
-    assert got_ratio.view(np.uint32) == np.float32(ratio).view(np.uint32)
-    np.testing.assert_array_equal(bits(adp.b_folded).ravel(), want)
+    if np.isfinite(ratio):
+        adp = L.prepare_nvfp4_lora_adapter(lb, st, at)
+        finish()
+        assert adp.ratio.cpu().numpy()[0].view(np.uint32) == np.float32(ratio).view(np.uint32)
+        np.testing.assert_array_equal(bits(adp.b_folded).ravel(), want)
+    else:
+        with pytest.raises(ValueError):
+            L.prepare_nvfp4_lora_adapter(lb, st, at)
+        adp = L.prepare_nvfp4_lora_adapter(lb, torch.tensor([1.0], device="cuda"), at if alpha != 0 else
+                                           torch.tensor([1.0], device="cuda"))
+        at = adp.alpha
+        at.fill_(alpha)
     # in-place refold into the same adapter is bitwise the eager form
     adp.b_folded.fill_(1.0)
     adp.ratio.fill_(-5.0)
     L.prepare_nvfp4_lora_adapter(lb, st, at, out=adp)
     finish()
     np.testing.assert_array_equal(bits(adp.b_folded).ravel(), want)
-    assert adp.ratio.cpu().numpy()[0].view(np.uint32) == np.float32(ratio).view(np.uint32)
+    got = adp.ratio.cpu().numpy()[0]
+    assert got.view(np.uint32) == np.float32(ratio).view(np.uint32) or (np.isnan(got) and np.isnan(ratio))
 
 
 def test_eager_prepare_refuses_alpha_zero_and_nonfinite_ratio():
@@ -157,8 +167,11 @@ def test_exact_regime_bitwise(M, N, K):
 # tolerance parity over shapes with several tiles and ragged tails
 # ---------------------------------------------------------------------------------------
 
+# M <= 32 runs the decode kernel (split-K cluster sizes 1, 2, 4, 8 below); larger M the tiled one
 SHAPES = [(1, 8, 256, 8), (16, 4096, 256, 64), (200, 300, 512, 16), (130, 1000, 768, 72),
-          (257, 129, 1024, 128), (384, 384, 2048, 32), (128, 256, 256, 16), (5, 100, 256, 24)]
+          (257, 129, 1024, 128), (384, 384, 2048, 32), (128, 256, 256, 16), (5, 100, 256, 24),
+          (3, 256, 2048, 16), (32, 1000, 1024, 128), (20, 9000, 512, 8), (16, 4096, 4096, 64),
+          (33, 520, 512, 40)]
 
 
 @pytest.mark.parametrize("M,N,K,r", SHAPES)
