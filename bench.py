@@ -58,6 +58,21 @@ def algorithmic(c):
     return nbytes, 2 * M * N * K, 2 * M * N * r
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The slowest rank's time: every rank contributes its own, all receive the maximum."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job(per_rank_value: float, world: int) -> float:
+    """Weak scaling: every rank processes the same amount of work in the (max-over-ranks) time,
+    so the whole-job throughput is the per-rank throughput times the number of ranks."""
+    return per_rank_value * world
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -230,9 +245,7 @@ def run_ours(args, rank, world, device):
     ms = start.elapsed_time(end)
     L.nvfp4lora_device_status(stream)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, device)
     ms_step = ms / K_steps
 
     # end to end through the public API with host buffers: per step, the activation-side
@@ -442,11 +455,11 @@ def main():
     e2e = res["e2e"]
     e2e_val, e2e_unit = metric_value(c, res["nbytes"], res["flops"], e2e["ms_step"] * 1.0)
     line = {
-        "metric": METRIC, "value": value * world, "unit": unit, "n_gpus": world, "steps": res["K"],
+        "metric": METRIC, "value": whole_job(value, world), "unit": unit, "n_gpus": world, "steps": res["K"],
         "warmup": res["W"], "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3 -> fp32) + bf16 LoRA", "data": "synthetic",
         "config": config_block(args, c), "roofline": roof, "clocks": res["clocks"],
-        "e2e": {"value": e2e_val * world, "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
+        "e2e": {"value": whole_job(e2e_val, world), "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"],
                 "note": "per step: a, a_sf, d host->device (pinned), call, out device->host; weights resident"},
         "gpu_launches": res["launches"],

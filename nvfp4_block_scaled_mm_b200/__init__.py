@@ -25,7 +25,7 @@ from typing import Optional
 
 import torch
 
-from .build import LIB_PATH
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4lora.so")
 
 __all__ = [
     "StaleAdapterError", "PreparedNvFp4LoraAdapter", "mm_nvfp4_lora", "prepare_nvfp4_lora_adapter",

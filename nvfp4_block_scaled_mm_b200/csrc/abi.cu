@@ -186,7 +186,7 @@ nvfp4lora_status check_base(const uint8_t* a, const uint8_t* b, const uint8_t* a
 // ---------------------------------------------------------------------------------------
 
 constexpr int kBN = 128;
-constexpr int kStages = 6;
+constexpr int kStages = 5;
 
 template <Mode MODE>
 nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
@@ -202,15 +202,20 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     constexpr int smem = GemmSmem<kBN, kStages>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
-    CUtensorMap tm_a, tm_b, tm_d, tm_lb;
+    const bool tma_store = (N % 8) == 0;
+    CUtensorMap tm_a, tm_b, tm_d, tm_lb, tm_out;
     std::memset(&tm_d, 0, sizeof(tm_d));
     std::memset(&tm_lb, 0, sizeof(tm_lb));
+    std::memset(&tm_out, 0, sizeof(tm_out));
     if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) != NVFP4LORA_OK) return st;
     if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, kBN)) != NVFP4LORA_OK) return st;
     if (MODE != Mode::Off) {
         if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128)) != NVFP4LORA_OK) return st;
         if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, kBN)) != NVFP4LORA_OK) return st;
     }
+    if (tma_store &&
+        (st = encode_2d(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 128)) != NVFP4LORA_OK)
+        return st;
 
     GemmArgs args;
     args.a_sf = a_sf;
@@ -231,6 +236,8 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     args.k_stages = (int)(K / 256);
     args.sf_atoms_k = (int)(K / 64);
     args.sf_row_blocks_b = (int)((N + 127) / 128);
+    args.tma_store = tma_store ? 1 : 0;
+    args.bias_vec = (bias != nullptr && aligned(bias, 16) && N % 8 == 0) ? 1 : 0;
 
     const int grid = (int)std::min<int64_t>(tiles, info->sms);
     cudaLaunchConfig_t cfg = {};
@@ -238,7 +245,7 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     cfg.blockDim = dim3(kGemmThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, args);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_out, args);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
     return NVFP4LORA_OK;
 }
@@ -248,12 +255,11 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
 // ---------------------------------------------------------------------------------------
 
 constexpr int kDecodeMaxM = 32;
-constexpr int kDecodeStages = 8;
 
 // Largest cluster split S in {8, 4, 2, 1} that keeps n_tiles * S CTAs within one wave and
 // divides the K stages.
 int decode_splits(int n_tiles, int k_stages, int sms) {
-    for (int s = 8; s > 1; s >>= 1)
+    for (int s = kDecodeMaxSplits; s > 1; s >>= 1)
         if (k_stages % s == 0 && (int64_t)n_tiles * s <= sms) return s;
     return 1;
 }
@@ -264,8 +270,9 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
                                   const uint16_t* lb, int64_t r, const uint16_t* bias, uint16_t* out,
                                   int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     nvfp4lora_status st;
-    auto kernel = nvfp4_decode_kernel<MT, kDecodeStages, MODE>;
-    constexpr int smem = DecodeSmem<MT, kDecodeStages>::DYN_BYTES;
+    constexpr int STAGES = (MT == 16) ? 6 : 4;   // leaves room for the peers' partials
+    auto kernel = nvfp4_decode_kernel<MT, STAGES, MODE>;
+    constexpr int smem = DecodeSmem<MT, STAGES>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
     CUtensorMap tm_a, tm_b, tm_d, tm_lb;

@@ -6,14 +6,15 @@
 //     its N side holds the MT (16 or 32) token rows m (a, a_sf, d); the fp32 accumulator in
 //     TMEM is out^T for one 128-column slice of out;
 //   * split-K over a thread-block cluster: the S CTAs of a cluster each stream K/S of the
-//     weights; CTA rank 0 additionally computes the LoRA term into its own TMEM region;
-//     ranks 1..S-1 park their fp32 partials in shared memory and rank 0 sums them in rank
-//     order through distributed shared memory (fixed order, so the result is deterministic),
-//     then applies the epilogue and the single bf16 rounding;
+//     weights.  Ranks 1..S-1 push their fp32 partials straight from registers into rank 0's
+//     shared memory (remote stores, then a releasing remote mbarrier arrival) and exit; rank 0
+//     sums them in rank order (so the result is deterministic), adds the LoRA term it computed
+//     into its own TMEM region, applies the epilogue and the single bf16 rounding;
 //   * the raw combine is v = alpha*acc; v = fma(s, lacc, v); v += bias; the prepared combine
 //     adds the folded LoRA term to the fully reduced base accumulator, then v = alpha*acc
 //     (+ bias) -- base first, LoRA after, alpha once.
-// All cross-CTA waits are bounded mbarrier waits; no global scratch memory is used.
+// The producer starts streaming weights as soon as the mbarriers exist; TMEM allocation and the
+// cluster barrier happen off that path.  All waits are bounded; no global scratch memory is used.
 #pragma once
 
 #include <cstdint>
@@ -40,24 +41,27 @@ struct DecodeArgs {
     int sf_row_blocks_b;     // ceil(N / 128)
 };
 
+constexpr int kDecodeMaxSplits = 8;
+
 template <int MT, int STAGES>
 struct DecodeSmem {
     static constexpr int W_BYTES = 128 * 128;          // weight tile: 128 rows x 128 bytes
     static constexpr int X_BYTES = MT * 128;           // token tile: MT rows x 128 bytes
     static constexpr int SF_BYTES = 4 * 512;           // 4 scale atoms (one 128-row block)
+    static constexpr int PART_SLOT = 128 * MT * 4;     // one peer's fp32 partial, [128][MT]
     static constexpr int W_OFF = 0;
     static constexpr int X_OFF = W_OFF + STAGES * W_BYTES;
     static constexpr int SFW_OFF = X_OFF + STAGES * X_BYTES;
     static constexpr int SFX_OFF = SFW_OFF + STAGES * SF_BYTES;
-    static constexpr int PART_OFF = SFX_OFF + STAGES * SF_BYTES;     // fp32 [MT][128] partial
-    static constexpr int PART_BYTES = MT * 128 * 4;
-    static constexpr int BAR_OFF = PART_OFF + PART_BYTES;
-    // full[S], empty[S], tmem_full, drain, parts_full, release
-    static constexpr int NUM_BARS = 2 * STAGES + 4;
+    static constexpr int PART_OFF = SFX_OFF + STAGES * SF_BYTES;   // rank 0: peers' partials
+    static constexpr int BAR_OFF = PART_OFF + (kDecodeMaxSplits - 1) * PART_SLOT;
+    // full[S], empty[S], tmem_full, drain, parts_full
+    static constexpr int NUM_BARS = 2 * STAGES + 3;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int DYN_BYTES = TOTAL + 1024;
     static_assert(X_BYTES % 1024 == 0, "token tiles must stay 1024-byte aligned");
+    static_assert(DYN_BYTES <= 232448, "decode shared-memory plan exceeds 227 KB");
 };
 
 template <int MT, int STAGES>
@@ -74,6 +78,8 @@ struct DecodeTmem {
     static_assert(USED <= 512, "TMEM plan exceeds 512 columns");
 };
 
+constexpr uint32_t kDecodeTmemBarrier = 2;   // named barrier: MMA warp + epilogue warps (160)
+
 template <int MT, int STAGES, Mode MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -81,7 +87,7 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                     const DecodeArgs args) {
     using L = DecodeSmem<MT, STAGES>;
     using T = DecodeTmem<MT, STAGES>;
-    static_assert(MT % 16 == 0 && MT <= 64, "MT must be 16, 32, 48 or 64");
+    static_assert(MT % 16 == 0 && MT <= 32, "MT must be 16 or 32");
     constexpr uint32_t IDESC_F4 = idesc_nvf4(MT);
     constexpr uint32_t IDESC_BF16 = idesc_bf16(MT);
 
@@ -92,8 +98,7 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
     uint64_t* empty = full + STAGES;
     uint64_t* tmem_full = empty + STAGES;
     uint64_t* drain = tmem_full + 1;
-    uint64_t* parts_full = drain + 1;    // rank 0: all peers' partials are parked
-    uint64_t* release = parts_full + 1;  // ranks > 0: rank 0 has finished reading this CTA
+    uint64_t* parts_full = drain + 1;    // rank 0: every peer's partial has landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
     float* part = reinterpret_cast<float*>(smem + L::PART_OFF);
@@ -101,81 +106,67 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_blk = blockIdx.x;
-    const uint32_t rank = (args.splits > 1) ? cluster_rank() : 0u;
+    const bool clustered = args.splits > 1;
+    const uint32_t rank = clustered ? cluster_rank() : 0u;
     const int k0 = (int)rank * args.stages_per_split;
+    const int base_items = args.stages_per_split;
 
-    float lora_s = 0.0f;
-    bool lora_on = false;
-    if constexpr (MODE != Mode::Off) {
-        lora_s = *args.scale;
-        lora_on = (lora_s != 0.0f) && rank == 0;
-    }
-    const int lora_chunks = lora_on ? (args.r + 63) / 64 : 0;
-    const int items = args.stages_per_split + lora_chunks;
+    // The zero-adapter decision (rank 0 only) reads a device scalar; each role issues the load
+    // early and consumes it once its base work is under way.
+    auto lora_scale_value = [&]() -> float {
+        if constexpr (MODE != Mode::Off) return rank == 0 ? *args.scale : 0.0f;
+        return 0.0f;
+    };
 
     if (threadIdx.x == 0) {
+        prefetch_tensor_map(&tm_b);
+        prefetch_tensor_map(&tm_a);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(tmem_full, 1);
         mbar_init(drain, 1);
-        mbar_init(parts_full, 128 * (args.splits - 1) > 0 ? 128 * (args.splits - 1) : 1);
-        mbar_init(release, 128);
+        mbar_init(parts_full, clustered ? 128 * (args.splits - 1) : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensor_map(&tm_a);
-        prefetch_tensor_map(&tm_b);
-        if (lora_on) {
-            prefetch_tensor_map(&tm_d);
-            prefetch_tensor_map(&tm_lb);
-        }
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, T::ALLOC);
-        tmem_relinquish();
-    }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
-    if (args.splits > 1) {
-        // every CTA's barriers must be initialised before any peer arrives on them
-        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    }
-    const uint32_t tmem = *tmem_slot;
+    if (clustered) cluster_arrive();   // this CTA's barriers exist; waited on before remote access
 
     if (warp == 0) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
+            const float sv = lora_scale_value();
             int stage = 0;
             uint32_t phase = 0, filled = 0, filled_parity = 0;
             bool ok = true;
-            for (int it = 0; it < items; ++it) {
-                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                const bool is_lora = it < lora_chunks;       // LoRA chunks first (rank 0 only)
-                uint8_t* sw = smem + L::W_OFF + stage * L::W_BYTES;
-                uint8_t* sx = smem + L::X_OFF + stage * L::X_BYTES;
-                if (is_lora) {
-                    mbar_arrive_expect_tx(&full[stage], L::W_BYTES + L::X_BYTES);
-                    tma_load_2d(sw, &tm_lb, &full[stage], it * 64, n_blk * 128);
-                    tma_load_2d(sx, &tm_d, &full[stage], it * 64, 0);
-                } else {
-                    const int kb = k0 + (it - lora_chunks);
-                    const bool sfw_ok = n_blk < args.sf_row_blocks_b;
-                    mbar_arrive_expect_tx(&full[stage], L::W_BYTES + L::X_BYTES + 2048 + (sfw_ok ? 2048 : 0));
-                    tma_load_2d(sw, &tm_b, &full[stage], kb * 128, n_blk * 128);
-                    tma_load_2d(sx, &tm_a, &full[stage], kb * 128, 0);
-                    if (sfw_ok)
-                        bulk_load(smem + L::SFW_OFF + stage * L::SF_BYTES,
-                                  args.b_sf + ((size_t)n_blk * args.sf_atoms_k + kb * 4) * 512, 2048, &full[stage]);
-                    bulk_load(smem + L::SFX_OFF + stage * L::SF_BYTES, args.a_sf + (size_t)kb * 4 * 512, 2048,
-                              &full[stage]);
-                }
+            auto next_stage = [&]() {
                 filled |= 1u << stage;
                 filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            };
+            for (int it = 0; ok && it < base_items; ++it) {
+                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                const int kb = k0 + it;
+                const bool sfw_ok = n_blk < args.sf_row_blocks_b;
+                mbar_arrive_expect_tx(&full[stage], L::W_BYTES + L::X_BYTES + 2048 + (sfw_ok ? 2048 : 0));
+                tma_load_2d(smem + L::W_OFF + stage * L::W_BYTES, &tm_b, &full[stage], kb * 128, n_blk * 128);
+                if (sfw_ok)
+                    bulk_load(smem + L::SFW_OFF + stage * L::SF_BYTES,
+                              args.b_sf + ((size_t)n_blk * args.sf_atoms_k + kb * 4) * 512, 2048, &full[stage]);
+                tma_load_2d(smem + L::X_OFF + stage * L::X_BYTES, &tm_a, &full[stage], kb * 128, 0);
+                bulk_load(smem + L::SFX_OFF + stage * L::SF_BYTES, args.a_sf + (size_t)kb * 4 * 512, 2048,
+                          &full[stage]);
+                next_stage();
+            }
+            const int chunks = (sv != 0.0f) ? (args.r + 63) / 64 : 0;   // LoRA after the base stages
+            for (int c = 0; ok && c < chunks; ++c) {
+                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                mbar_arrive_expect_tx(&full[stage], L::W_BYTES + L::X_BYTES);
+                tma_load_2d(smem + L::W_OFF + stage * L::W_BYTES, &tm_lb, &full[stage], c * 64, n_blk * 128);
+                tma_load_2d(smem + L::X_OFF + stage * L::X_BYTES, &tm_d, &full[stage], c * 64, 0);
+                next_stage();
             }
             if (!ok || *abort_flag) {
                 for (int s = 0; s < STAGES; ++s)
@@ -184,38 +175,53 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
+        tmem_alloc(tmem_slot, T::ALLOC);
+        tmem_relinquish();
+        tc_fence_before();
+        named_barrier_sync(kDecodeTmemBarrier, 160);   // hands the TMEM address to the epilogue
+        tc_fence_after();
+        const uint32_t tmem = *tmem_slot;
         if (lane == 0) {
+            const float sv = lora_scale_value();
+            if (MODE != Mode::Off && rank == 0) {
+                prefetch_tensor_map(&tm_d);
+                prefetch_tensor_map(&tm_lb);
+            }
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int it = 0; it < items; ++it) {
+            for (int it = 0; ok && it < base_items; ++it) {
                 if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const bool is_lora = it < lora_chunks;
                 const uint32_t w_addr = smem_u32(smem + L::W_OFF + stage * L::W_BYTES);
                 const uint32_t x_addr = smem_u32(smem + L::X_OFF + stage * L::X_BYTES);
-                if (is_lora) {
-                    const int rem = args.r - it * 64;
-                    const int ksteps = rem >= 64 ? 4 : (rem + 15) / 16;
-                    for (int j = 0; j < ksteps; ++j)
-                        tc_mma_bf16(tmem + T::LACC, sdesc_sw128(w_addr + j * 32), sdesc_sw128(x_addr + j * 32),
-                                    IDESC_BF16, (it > 0 || j > 0) ? 1u : 0u);
-                } else {
-                    const int kl = it - lora_chunks;
-                    const uint32_t sfw_t = tmem + T::SF0 + stage * T::STAGE_COLS;
-                    const uint32_t sfx_t = sfw_t + T::SFW_COLS;
-                    const uint32_t sfw_s = smem_u32(smem + L::SFW_OFF + stage * L::SF_BYTES);
-                    const uint32_t sfx_s = smem_u32(smem + L::SFX_OFF + stage * L::SF_BYTES);
+                const uint32_t sfw_t = tmem + T::SF0 + stage * T::STAGE_COLS;
+                const uint32_t sfx_t = sfw_t + T::SFW_COLS;
+                const uint32_t sfw_s = smem_u32(smem + L::SFW_OFF + stage * L::SF_BYTES);
+                const uint32_t sfx_s = smem_u32(smem + L::SFX_OFF + stage * L::SF_BYTES);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tc_copy_scale_atom(sfw_t + 4 * j, sdesc_scale_atom(sfw_s + j * 512));
-                        tc_copy_scale_atom(sfx_t + 4 * j, sdesc_scale_atom(sfx_s + j * 512));
-                    }
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tc_mma_nvf4(tmem + T::ACC, sdesc_sw128(w_addr + j * 32), sdesc_sw128(x_addr + j * 32),
-                                    IDESC_F4, sfw_t + 4 * j, sfx_t + 4 * j, (kl > 0 || j > 0) ? 1u : 0u);
+                for (int j = 0; j < 4; ++j) {
+                    tc_copy_scale_atom(sfw_t + 4 * j, sdesc_scale_atom(sfw_s + j * 512));
+                    tc_copy_scale_atom(sfx_t + 4 * j, sdesc_scale_atom(sfx_s + j * 512));
                 }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    tc_mma_nvf4(tmem + T::ACC, sdesc_sw128(w_addr + j * 32), sdesc_sw128(x_addr + j * 32),
+                                IDESC_F4, sfw_t + 4 * j, sfx_t + 4 * j, (it > 0 || j > 0) ? 1u : 0u);
+                tc_commit(&empty[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+            const int chunks = (sv != 0.0f) ? (args.r + 63) / 64 : 0;
+            for (int c = 0; ok && c < chunks; ++c) {
+                if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t w_addr = smem_u32(smem + L::W_OFF + stage * L::W_BYTES);
+                const uint32_t x_addr = smem_u32(smem + L::X_OFF + stage * L::X_BYTES);
+                const int rem = args.r - c * 64;
+                const int ksteps = rem >= 64 ? 4 : (rem + 15) / 16;
+                for (int j = 0; j < ksteps; ++j)
+                    tc_mma_bf16(tmem + T::LACC, sdesc_sw128(w_addr + j * 32), sdesc_sw128(x_addr + j * 32),
+                                IDESC_BF16, (c > 0 || j > 0) ? 1u : 0u);
                 tc_commit(&empty[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
@@ -232,6 +238,14 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
         const int nl = q * 32 + lane;                 // weight row within the tile = TMEM lane
         const int n = n_blk * 128 + nl;               // output column
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const float lora_s = lora_scale_value();
+        const bool lora_on = (lora_s != 0.0f);        // false on ranks > 0
+        const float alpha = (rank == 0) ? *args.alpha : 0.0f;
+        const float bias_v = (rank == 0 && args.bias != nullptr && n < args.N)
+                                 ? __uint_as_float((uint32_t)__ldg(args.bias + n) << 16) : 0.0f;
+        named_barrier_sync(kDecodeTmemBarrier, 160);
+        tc_fence_after();
+        const uint32_t tmem = *tmem_slot;
         bool ok = mbar_wait(tmem_full, 0, abort_flag);
         float acc[MT];
         if (ok) {
@@ -246,12 +260,14 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
             }
         }
         if (rank != 0) {
-            // park the partial and tell rank 0; wait until rank 0 has read it
+            // push the partial into rank 0's slot (rank - 1), then signal it
+            cluster_wait();
             if (ok) {
+                const uint32_t dst = map_to_rank(smem_u32(part + (size_t)(rank - 1) * 128 * MT + nl * MT), 0);
 #pragma unroll
-                for (int m = 0; m < MT; ++m) part[m * 128 + nl] = acc[m];
+                for (int m = 0; m < MT; m += 4)
+                    st_cluster_v4(dst + m * 4, acc[m], acc[m + 1], acc[m + 2], acc[m + 3]);
                 mbar_arrive_remote(map_to_rank(smem_u32(parts_full), 0));
-                mbar_wait_cluster(release, 0, abort_flag);
             }
         } else if (ok) {
             float lac[MT];
@@ -265,46 +281,51 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                     for (int i = 0; i < 16; ++i) lac[c * 16 + i] = __uint_as_float(v[i]);
                 }
             }
-            if (args.splits > 1) {
+            if (clustered) {
+                cluster_wait();
                 ok = mbar_wait_cluster(parts_full, 0, abort_flag);
                 if (ok) {
-                    const uint32_t local = smem_u32(part) + (uint32_t)nl * 4u;
                     for (int pr = 1; pr < args.splits; ++pr) {
-                        const uint32_t remote = map_to_rank(local, (uint32_t)pr);
+                        const float4* src =
+                            reinterpret_cast<const float4*>(part + (size_t)(pr - 1) * 128 * MT + nl * MT);
 #pragma unroll
-                        for (int m = 0; m < MT; ++m) acc[m] = __fadd_rn(acc[m], ld_cluster_f32(remote + m * 512u));
-                    }
-                    for (int pr = 1; pr < args.splits; ++pr)
-                        mbar_arrive_remote(map_to_rank(smem_u32(release), (uint32_t)pr));
-                }
-            }
-            if (ok) {
-                const float alpha = *args.alpha;
-                const float bias_v = (args.bias != nullptr && n < args.N)
-                                         ? __uint_as_float((uint32_t)__ldg(args.bias + n) << 16) : 0.0f;
-                if (n < args.N) {
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        float a = acc[m];
-                        if (MODE == Mode::Prepared && lora_on) a = __fadd_rn(a, lac[m]);
-                        float x = __fmul_rn(alpha, a);
-                        if (MODE == Mode::Raw && lora_on) x = __fmaf_rn(lora_s, lac[m], x);
-                        if (args.bias != nullptr) x = __fadd_rn(x, bias_v);
-                        if (m < args.M) {
-                            __nv_bfloat16 h = __float2bfloat16_rn(x);
-                            args.out[(size_t)m * args.N + n] = *reinterpret_cast<uint16_t*>(&h);
+                        for (int m = 0; m < MT; m += 4) {
+                            const float4 w = src[m / 4];
+                            acc[m] = __fadd_rn(acc[m], w.x);
+                            acc[m + 1] = __fadd_rn(acc[m + 1], w.y);
+                            acc[m + 2] = __fadd_rn(acc[m + 2], w.z);
+                            acc[m + 3] = __fadd_rn(acc[m + 3], w.w);
                         }
                     }
                 }
             }
+            if (ok && n < args.N) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    float a = acc[m];
+                    if (MODE == Mode::Prepared && lora_on) a = __fadd_rn(a, lac[m]);
+                    float x = __fmul_rn(alpha, a);
+                    if (MODE == Mode::Raw && lora_on) x = __fmaf_rn(lora_s, lac[m], x);
+                    if (args.bias != nullptr) x = __fadd_rn(x, bias_v);
+                    if (m < args.M) {
+                        __nv_bfloat16 h = __float2bfloat16_rn(x);
+                        args.out[(size_t)m * args.N + n] = *reinterpret_cast<uint16_t*>(&h);
+                    }
+                }
+            }
+        } else if (clustered) {
+            cluster_wait();
         }
     }
+    // Every thread arrived on the cluster barrier once; the ones that did not need it wait here,
+    // so each thread completes exactly one arrive/wait pair.
+    if (clustered && warp < 2) cluster_wait();
 
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, T::ALLOC);
+        tmem_dealloc(*tmem_slot, T::ALLOC);
     }
 }
 

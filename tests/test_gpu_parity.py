@@ -387,3 +387,16 @@ def test_cfg4_adapter_switch_shapes(M, r):
         ci = torch.from_numpy(cols).cuda()
         check_close(out[ri][:, ci], y, what=f"cfg4 raw M{M} r{r}")
         check_close(outp[ri][:, ci], yp, what=f"cfg4 prepared M{M} r{r}")
+
+
+@pytest.mark.parametrize("M,N", [(200, 512), (16, 512)])
+def test_bias_not_16_byte_aligned(M, N):
+    """A bias view that starts 2 bytes into its storage takes the element-wise bias path."""
+    p = make_problem(M, N, 512, 16, seed=12, alpha=2.0 ** -6, lora_scale=1.0, bias=True)
+    x = Dev(p)
+    store = torch.empty(N + 8, dtype=torch.bfloat16, device="cuda")
+    store[1:N + 1] = x.bias
+    x.bias = store[1:N + 1]
+    out = run_raw(x, x.lora_scale)
+    finish()
+    check_close(out, oracle_raw(p, host_arrays(p), 1.0), what="unaligned bias")
