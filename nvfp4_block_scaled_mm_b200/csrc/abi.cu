@@ -185,8 +185,7 @@ nvfp4lora_status check_base(const uint8_t* a, const uint8_t* b, const uint8_t* a
 // GEMM launch
 // ---------------------------------------------------------------------------------------
 
-constexpr int kBN = 128;
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 
 template <Mode MODE>
 nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
@@ -198,24 +197,19 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     nvfp4lora_status st = device_info(&dev, &info);
     if (st != NVFP4LORA_OK) return st;
 
-    auto kernel = nvfp4_gemm_kernel<kBN, kStages, MODE>;
-    constexpr int smem = GemmSmem<kBN, kStages>::DYN_BYTES;
+    auto kernel = nvfp4_gemm_kernel<kStages, MODE>;
+    constexpr int smem = GemmSmem<kStages>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
-    const bool tma_store = (N % 8) == 0;
-    CUtensorMap tm_a, tm_b, tm_d, tm_lb, tm_out;
+    CUtensorMap tm_a, tm_b, tm_d, tm_lb;
     std::memset(&tm_d, 0, sizeof(tm_d));
     std::memset(&tm_lb, 0, sizeof(tm_lb));
-    std::memset(&tm_out, 0, sizeof(tm_out));
-    if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) != NVFP4LORA_OK) return st;
-    if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, kBN)) != NVFP4LORA_OK) return st;
+    if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, kTileM)) != NVFP4LORA_OK) return st;
+    if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, kTileN)) != NVFP4LORA_OK) return st;
     if (MODE != Mode::Off) {
-        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128)) != NVFP4LORA_OK) return st;
-        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, kBN)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, kTileM)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, kTileN)) != NVFP4LORA_OK) return st;
     }
-    if (tma_store &&
-        (st = encode_2d(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 128)) != NVFP4LORA_OK)
-        return st;
 
     GemmArgs args;
     args.a_sf = a_sf;
@@ -228,16 +222,15 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     args.N = (int)N;
     args.K = (int)K;
     args.r = (int)r;
-    args.m_tiles = (int)((M + 127) / 128);
-    args.n_tiles = (int)((N + kBN - 1) / kBN);
+    args.m_tiles = (int)((M + kTileM - 1) / kTileM);
+    args.n_tiles = (int)((N + kTileN - 1) / kTileN);
     const int64_t tiles = (int64_t)args.m_tiles * args.n_tiles;
     if (tiles > INT32_MAX) return fail(NVFP4LORA_ERR_INVALID_ARG, "too many output tiles (M x N too large)");
     args.num_tiles = (int)tiles;
     args.k_stages = (int)(K / 256);
     args.sf_atoms_k = (int)(K / 64);
     args.sf_row_blocks_b = (int)((N + 127) / 128);
-    args.tma_store = tma_store ? 1 : 0;
-    args.bias_vec = (bias != nullptr && aligned(bias, 16) && N % 8 == 0) ? 1 : 0;
+    args.vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16))) ? 1 : 0;
 
     const int grid = (int)std::min<int64_t>(tiles, info->sms);
     cudaLaunchConfig_t cfg = {};
@@ -245,7 +238,12 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     cfg.blockDim = dim3(kGemmThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_out, args);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, args);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
     return NVFP4LORA_OK;
 }
@@ -304,17 +302,20 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(args.n_tiles, args.splits);
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(kDecodeThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (args.splits > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 1;
-        attr[0].val.clusterDim.y = args.splits;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 1;
+        attr[1].val.clusterDim.y = args.splits;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
     }
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, args);
     if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");

@@ -30,6 +30,8 @@ constexpr int kFoldThreads = 256;
 __global__ void __launch_bounds__(kFoldThreads)
 fold_kernel(const uint16_t* lora_b, const float* lora_scale, const float* alpha,
             uint16_t* b_folded, float* ratio_out, int64_t groups) {
+    // Let a dependent GEMM begin its prologue; it still waits for this grid before reading.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const float ratio = __fdiv_rn(*lora_scale, *alpha);
     if (blockIdx.x == 0 && threadIdx.x == 0) *ratio_out = ratio;
     const uint4* src = reinterpret_cast<const uint4*>(lora_b);

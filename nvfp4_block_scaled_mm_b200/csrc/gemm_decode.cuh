@@ -42,6 +42,7 @@ struct DecodeArgs {
 };
 
 constexpr int kDecodeMaxSplits = 8;
+constexpr int kDecodeThreads = 192;       // producer, MMA, 4 epilogue warps
 
 template <int MT, int STAGES>
 struct DecodeSmem {
@@ -81,7 +82,7 @@ struct DecodeTmem {
 constexpr uint32_t kDecodeTmemBarrier = 2;   // named barrier: MMA warp + epilogue warps (160)
 
 template <int MT, int STAGES, Mode MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kDecodeThreads, 1)
 nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_lb,
                     const DecodeArgs args) {
@@ -133,10 +134,22 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
     }
     __syncthreads();
     if (clustered) cluster_arrive();   // this CTA's barriers exist; waited on before remote access
+    // Programmatic dependent launch: the next kernel on the stream may start its own prologue
+    // now; every access to memory another kernel may write comes after grid_dependency_wait().
+    grid_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
+            // Warm L2 with this CTA's weight tiles while the previous kernel finishes (a prefetch
+            // changes no data, so it may precede the dependency wait).
+            for (int it = 0; it < base_items; ++it) {
+                const int kb = k0 + it;
+                tma_prefetch_l2_2d(&tm_b, kb * 128, n_blk * 128);
+                if (n_blk < args.sf_row_blocks_b)
+                    bulk_prefetch_l2(args.b_sf + ((size_t)n_blk * args.sf_atoms_k + kb * 4) * 512, 2048);
+            }
+            grid_dependency_wait();
             const float sv = lora_scale_value();
             int stage = 0;
             uint32_t phase = 0, filled = 0, filled_parity = 0;
@@ -182,6 +195,7 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
         tc_fence_after();
         const uint32_t tmem = *tmem_slot;
         if (lane == 0) {
+            grid_dependency_wait();
             const float sv = lora_scale_value();
             if (MODE != Mode::Off && rank == 0) {
                 prefetch_tensor_map(&tm_d);
@@ -238,6 +252,7 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
         const int nl = q * 32 + lane;                 // weight row within the tile = TMEM lane
         const int n = n_blk * 128 + nl;               // output column
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        grid_dependency_wait();
         const float lora_s = lora_scale_value();
         const bool lora_on = (lora_s != 0.0f);        // false on ranks > 0
         const float alpha = (rank == 0) ? *args.alpha : 0.0f;

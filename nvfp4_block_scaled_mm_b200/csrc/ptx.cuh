@@ -352,3 +352,34 @@ __device__ __forceinline__ void cluster_wait() {
 }
 
 }  // namespace nvfp4lora
+
+namespace nvfp4lora {
+
+// ------------------------------------------------------------------------------------
+// programmatic dependent launch and L2 prefetch
+// ------------------------------------------------------------------------------------
+
+// Block until the grids this one depends on (launched before it on the stream) have completed
+// and their memory is visible.  A no-op when the kernel was launched without the programmatic
+// serialization attribute.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next grid on the stream to be scheduled (its own griddepcontrol.wait still waits
+// for this grid to finish).
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Pull a 2-D tensor tile into L2 without writing shared memory (no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+                 ::"l"(map), "r"(x), "r"(y) : "memory");
+}
+
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+}  // namespace nvfp4lora
