@@ -93,6 +93,9 @@ nvfp4lora_status ensure_smem_attr(DeviceInfo* info, Kernel kernel, int smem) {
     const void* key = reinterpret_cast<const void*>(kernel);
     if (info->smem_attr_set.count(key)) return NVFP4LORA_OK;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the whole unified L1 / shared array as shared memory, so co-resident CTAs fit
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     info->smem_attr_set.insert(key);
     return NVFP4LORA_OK;
@@ -136,6 +139,24 @@ nvfp4lora_status encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataTy
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(NVFP4LORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return NVFP4LORA_OK;
+}
+
+// 3-D view of a row-major [rows, cols] uint8 matrix as (128-byte chunk, row, chunk index), used
+// to name one 128-row block across several K chunks in a single box (L2 prefetch only).
+nvfp4lora_status encode_rows_by_chunks(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                                       uint32_t box_rows, uint32_t box_chunks) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+    nvfp4lora_status st = get_encoder(&enc);
+    if (st != NVFP4LORA_OK) return st;
+    cuuint64_t dims[3] = {128, rows, cols / 128};
+    cuuint64_t strides[2] = {cols, 128};
+    cuuint32_t box[3] = {128, box_rows, box_chunks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NVFP4LORA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (CUresult %d)", (int)r);
     return NVFP4LORA_OK;
 }
 
@@ -254,10 +275,10 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
 
 constexpr int kDecodeMaxM = 32;
 
-// Largest cluster split S in {8, 4, 2, 1} that keeps n_tiles * S CTAs within one wave and
-// divides the K stages.
-int decode_splits(int n_tiles, int k_stages, int sms) {
-    for (int s = kDecodeMaxSplits; s > 1; s >>= 1)
+// Largest cluster split S <= max_s (a power of two) that keeps n_tiles * S CTAs within one wave
+// and divides the K stages.
+int decode_splits(int n_tiles, int k_stages, int sms, int max_s) {
+    for (int s = max_s; s > 1; s >>= 1)
         if (k_stages % s == 0 && (int64_t)n_tiles * s <= sms) return s;
     return 1;
 }
@@ -268,9 +289,11 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
                                   const uint16_t* lb, int64_t r, const uint16_t* bias, uint16_t* out,
                                   int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     nvfp4lora_status st;
-    constexpr int STAGES = (MT == 16) ? 6 : 4;   // leaves room for the peers' partials
-    auto kernel = nvfp4_decode_kernel<MT, STAGES, MODE>;
-    constexpr int smem = DecodeSmem<MT, STAGES>::DYN_BYTES;
+    // one CTA per SM; rank 0 keeps room for MAXS - 1 peers' partials
+    constexpr int STAGES = 4;
+    constexpr int MAXS = (MT == 16) ? 8 : 4;
+    auto kernel = nvfp4_decode_kernel<MT, STAGES, MAXS, MODE>;
+    constexpr int smem = DecodeSmem<MT, STAGES, MAXS>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
     CUtensorMap tm_a, tm_b, tm_d, tm_lb;
@@ -295,10 +318,15 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
     args.r = (int)r;
     args.n_tiles = (int)((N + 127) / 128);
     const int k_stages = (int)(K / 256);
-    args.splits = decode_splits(args.n_tiles, k_stages, info->sms);
+    args.splits = decode_splits(args.n_tiles, k_stages, info->sms, MAXS);
     args.stages_per_split = k_stages / args.splits;
     args.sf_atoms_k = (int)(K / 64);
     args.sf_row_blocks_b = (int)((N + 127) / 128);
+
+    CUtensorMap tm_b3;
+    // one prefetch box covers up to 8 chunks (128 KB, within the tensor-map box limit)
+    args.pf_chunks = std::min(args.stages_per_split, 8);
+    if ((st = encode_rows_by_chunks(&tm_b3, b, K / 2, N, 128, args.pf_chunks)) != NVFP4LORA_OK) return st;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(args.n_tiles, args.splits);
@@ -317,7 +345,7 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
         attr[1].val.clusterDim.z = 1;
         cfg.numAttrs = 2;
     }
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, args);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_b3, args);
     if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
     return NVFP4LORA_OK;
 }

@@ -78,15 +78,17 @@ struct GemmSmem {
 // used round-robin by the pipeline stages, and the raw path's 128-column LoRA accumulator.
 // tcgen05.cp and tcgen05.mma issued by one thread execute in issue order, so a slot is never
 // rewritten before the MMAs that read it have consumed it.
+template <Mode MODE>
 struct TmemPlan {
     static constexpr int ACC = 0;
     static constexpr int SF0 = kTileN;
     static constexpr int SFA_COLS = 4 * 4;                // 4 MMAs (K = 64 each) x 4 columns
     static constexpr int SFB_COLS = 4 * (kTileN / 32);    // 4 MMAs x 8 columns
     static constexpr int SLOT_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int NSF = 2;
-    static constexpr int LACC = SF0 + NSF * SLOT_COLS;    // 352
-    static constexpr int USED = LACC + 128;
+    // more slots let a stage's scale copies run further ahead of the MMAs still reading older slots
+    static constexpr int NSF = (MODE == Mode::Raw) ? 2 : 5;
+    static constexpr int LACC = SF0 + NSF * SLOT_COLS;    // raw path: 352
+    static constexpr int USED = (MODE == Mode::Raw) ? LACC + 128 : LACC;
     static constexpr int ALLOC = 512;
     static_assert(USED <= ALLOC, "TMEM plan exceeds 512 columns");
 };
@@ -102,7 +104,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_lb,
                   const GemmArgs args) {
     using L = GemmSmem<STAGES>;
-    using T = TmemPlan;
+    using T = TmemPlan<MODE>;
     constexpr uint32_t IDESC_F4 = idesc_nvf4(kTileN);
     constexpr uint32_t IDESC_BF16_FULL = idesc_bf16(kTileN);
     constexpr uint32_t IDESC_BF16_HALF = idesc_bf16(kTileN / 2);

@@ -205,6 +205,23 @@ __device__ __forceinline__ void tmem_load_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Warp-collective store of 32 columns from registers into this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_store_32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+        " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+          "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+          "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+// Wait until this thread's tcgen05.st stores have been performed.
+__device__ __forceinline__ void tmem_store_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------
 // descriptors
 // ------------------------------------------------------------------------------------
@@ -341,9 +358,11 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads
 namespace nvfp4lora {
 
 // Store 16 bytes into another CTA's shared memory (cluster address from map_to_rank).
-__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
+// Asynchronous store into another CTA's shared memory whose completion is counted, in bytes, on
+// that CTA's mbarrier (complete_tx): the receiver's wait on the barrier makes the data visible.
+__device__ __forceinline__ void st_async_v4(uint32_t caddr, float a, float b, float c, float d, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(cbar) : "memory");
 }
 
 // Split cluster barrier: every thread of every CTA arrives once, early; a thread that is about
@@ -381,6 +400,11 @@ __device__ __forceinline__ void grid_launch_dependents() {
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
     asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
                  ::"l"(map), "r"(x), "r"(y) : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t x, int32_t y, int32_t z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(map), "r"(x), "r"(y), "r"(z) : "memory");
 }
 
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
