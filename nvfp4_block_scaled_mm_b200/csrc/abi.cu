@@ -310,6 +310,7 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
     args.b_sf = b_sf;
     args.alpha = alpha;
     args.scale = scale;
+    args.lb = lb;
     args.bias = bias;
     args.out = out;
     args.M = (int)M;

@@ -37,6 +37,7 @@ struct DecodeArgs {
     const uint8_t* b_sf;
     const float* alpha;
     const float* scale;      // Raw: lora_scale; Prepared: ratio; Off: unused
+    const uint16_t* lb;      // lora_b (raw) or b_folded (prepared): an L2 prefetch hint only
     const uint16_t* bias;
     uint16_t* out;
     int M, N, K, r;
@@ -91,6 +92,7 @@ struct DecodeTmem {
 
 constexpr uint32_t kDecodeTmemBarrier = 2;   // named barrier: MMA warp + epilogue warps (160)
 constexpr uint32_t kDecodeEpilogueBarrier = 3;   // named barrier: the 4 epilogue warps (128)
+constexpr uint32_t kDecodeDeallocBarrier = 4;    // named barrier: MMA warp + epilogue warps (160)
 
 template <int MT, int STAGES, int MAXS, Mode MODE>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
@@ -169,6 +171,10 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
             if (n_blk < args.sf_row_blocks_b)
                 bulk_prefetch_l2(args.b_sf + ((size_t)n_blk * args.sf_atoms_k + k0 * 4) * 512,
                                  (uint32_t)min(base_items, 64) * 2048u);
+            // rank 0 computes the LoRA term: its 128 rows of lora_b / b_folded are contiguous
+            if (MODE != Mode::Off && rank == 0)
+                bulk_prefetch_l2(args.lb + (size_t)n_blk * 128 * args.r,
+                                 (uint32_t)(min(128, args.N - n_blk * 128) * args.r * 2));
             grid_dependency_wait();
             const float sv = lora_scale_value();   // consumed after the ring's first fill
             int stage = 0;
@@ -268,6 +274,10 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
             }
         }
         __syncwarp();
+        // TMEM goes back as soon as the epilogue warps hold the accumulators in registers
+        named_barrier_sync(kDecodeDeallocBarrier, 160);
+        tc_fence_after();
+        tmem_dealloc(tmem, T::ALLOC);
     } else {
         // ------------------------------- epilogue -----------------------------------
         const int q = warp & 3;
@@ -314,7 +324,7 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
             }
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, abort_flag));
-        float acc[MT];
+        float acc[MT], lac[MT];
         if (ok) {
             tc_fence_after();
 #pragma unroll
@@ -325,7 +335,19 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc[c * 16 + i] = __uint_as_float(v[i]);
             }
+            if (lora_on) {
+#pragma unroll
+                for (int c = 0; c < MT / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_load_16(tmem + lane_off + T::LACC + c * 16, v);
+                    tmem_load_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) lac[c * 16 + i] = __uint_as_float(v[i]);
+                }
+            }
         }
+        tc_fence_before();
+        named_barrier_arrive(kDecodeDeallocBarrier, 160);   // accumulators read: TMEM may go
         bool parts_seen = false;
         // a peer's partial slot is [MT/4][128] float4: lane-consecutive 16-byte accesses
         if (rank != 0) {
@@ -338,17 +360,6 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                     st_async_v4(dst + m * 128 * 4, acc[m], acc[m + 1], acc[m + 2], acc[m + 3], bar);
             }
         } else {
-            float lac[MT];
-            if (ok && lora_on) {
-#pragma unroll
-                for (int c = 0; c < MT / 16; ++c) {
-                    uint32_t v[16];
-                    tmem_load_16(tmem + lane_off + T::LACC + c * 16, v);
-                    tmem_load_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) lac[c * 16 + i] = __uint_as_float(v[i]);
-                }
-            }
             if (ok && clustered) {
                 ok = __all_sync(0xffffffffu, mbar_wait_cluster(parts_full, 0, abort_flag));
                 parts_seen = ok;
@@ -406,13 +417,6 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
     // Every thread arrived on the cluster barrier once; the ones that did not need it wait here,
     // so each thread completes exactly one arrive/wait pair.
     if (clustered && warp < 2) cluster_wait();
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(*tmem_slot, T::ALLOC);
-    }
 }
 
 }  // namespace nvfp4lora
