@@ -139,6 +139,10 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
         prefetch_tensor_map(&tm_b3);
         prefetch_tensor_map(&tm_b);
         prefetch_tensor_map(&tm_a);
+        if (MODE != Mode::Off && rank == 0) {
+            prefetch_tensor_map(&tm_lb);
+            prefetch_tensor_map(&tm_d);
+        }
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -176,7 +180,6 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                 bulk_prefetch_l2(args.lb + (size_t)n_blk * 128 * args.r,
                                  (uint32_t)(min(128, args.N - n_blk * 128) * args.r * 2));
             grid_dependency_wait();
-            const float sv = lora_scale_value();   // consumed after the ring's first fill
             int stage = 0;
             uint32_t phase = 0, filled = 0, filled_parity = 0;
             bool ok = true, lora_issued = false;
@@ -185,7 +188,18 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                 filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             };
-            const int first_fill = min(STAGES, base_items);
+            if (MODE != Mode::Off && rank == 0) {
+                // The LoRA operands first, into their own buffers: they were warmed into L2 before
+                // the dependency wait, so they land before the base tiles.  A zero scale (read
+                // later) skips the LoRA MMAs; only these reads remain.
+                const int chunks = (args.r + 63) / 64;
+                mbar_arrive_expect_tx(lora_full, chunks * (L::W_BYTES + L::X_BYTES));
+                for (int c = 0; c < chunks; ++c) {
+                    tma_load_2d(smem + L::LW_OFF + c * L::W_BYTES, &tm_lb, lora_full, c * 64, n_blk * 128);
+                    tma_load_2d(smem + L::LX_OFF + c * L::X_BYTES, &tm_d, lora_full, c * 64, 0);
+                }
+                lora_issued = true;
+            }
             for (int it = 0; ok && it < base_items; ++it) {
                 if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                 const int kb = k0 + it;
@@ -198,16 +212,6 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                 tma_load_2d(smem + L::W_OFF + stage * L::W_BYTES, &tm_b, &full[stage], kb * 128, n_blk * 128);
                 tma_load_2d(smem + L::X_OFF + stage * L::X_BYTES, &tm_a, &full[stage], kb * 128, 0);
                 next_stage();
-                if (it == first_fill - 1 && sv != 0.0f) {
-                    // the LoRA operands, into their own buffers (rank 0 only: sv is 0 elsewhere)
-                    const int chunks = (args.r + 63) / 64;
-                    mbar_arrive_expect_tx(lora_full, chunks * (L::W_BYTES + L::X_BYTES));
-                    for (int c = 0; c < chunks; ++c) {
-                        tma_load_2d(smem + L::LW_OFF + c * L::W_BYTES, &tm_lb, lora_full, c * 64, n_blk * 128);
-                        tma_load_2d(smem + L::LX_OFF + c * L::X_BYTES, &tm_d, lora_full, c * 64, 0);
-                    }
-                    lora_issued = true;
-                }
             }
             if (!ok || *abort_flag) {
                 for (int s = 0; s < STAGES; ++s)
@@ -215,8 +219,9 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                         mbar_wait(&sf_full[s], (filled_parity >> s) & 1u, nullptr);
                         mbar_wait(&full[s], (filled_parity >> s) & 1u, nullptr);
                     }
-                if (lora_issued) mbar_wait(lora_full, 0, nullptr);
             }
+            // the LoRA bytes land before the CTA can end, also when a zero scale skipped their MMAs
+            if (lora_issued) mbar_wait(lora_full, 0, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------- MMA issuer ---------------------------------
@@ -228,30 +233,10 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
         const uint32_t tmem = *tmem_slot;
         if (lane == 0) {
             grid_dependency_wait();
-            const float sv = lora_scale_value();
-            if (MODE != Mode::Off && rank == 0) {
-                prefetch_tensor_map(&tm_d);
-                prefetch_tensor_map(&tm_lb);
-            }
-            int stage = 0;
-            uint32_t phase = 0;
+            const float sv = (rank == 0) ? lora_scale_value() : 0.0f;
             bool ok = true;
-            for (int it = 0; ok && it < base_items; ++it) {
-                if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) { ok = false; break; }
-                if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t w_addr = smem_u32(smem + L::W_OFF + stage * L::W_BYTES);
-                const uint32_t x_addr = smem_u32(smem + L::X_OFF + stage * L::X_BYTES);
-                const uint32_t sfw_t = tmem + T::SF0 + stage * T::STAGE_COLS;
-                const uint32_t sfx_t = sfw_t + T::SFW_COLS;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    tc_mma_nvf4(tmem + T::ACC, sdesc_sw128(w_addr + j * 32), sdesc_sw128(x_addr + j * 32),
-                                IDESC_F4, sfw_t + 4 * j, sfx_t + 4 * j, (it > 0 || j > 0) ? 1u : 0u);
-                tc_commit(&empty[stage]);
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            }
-            if (ok && sv != 0.0f) {
+            if (sv != 0.0f) {
+                // the LoRA operands were issued first and land first: their MMAs go first
                 if (!mbar_wait(lora_full, 0, abort_flag)) ok = false;
                 if (ok) {
                     tc_fence_after();
@@ -266,6 +251,23 @@ nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_const
                                         IDESC_BF16, (c > 0 || j > 0) ? 1u : 0u);
                     }
                 }
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int it = 0; ok && it < base_items; ++it) {
+                if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t w_addr = smem_u32(smem + L::W_OFF + stage * L::W_BYTES);
+                const uint32_t x_addr = smem_u32(smem + L::X_OFF + stage * L::X_BYTES);
+                const uint32_t sfw_t = tmem + T::SF0 + stage * T::STAGE_COLS;
+                const uint32_t sfx_t = sfw_t + T::SFW_COLS;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    tc_mma_nvf4(tmem + T::ACC, sdesc_sw128(w_addr + j * 32), sdesc_sw128(x_addr + j * 32),
+                                IDESC_F4, sfw_t + 4 * j, sfx_t + 4 * j, (it > 0 || j > 0) ? 1u : 0u);
+                tc_commit(&empty[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
             if (ok) tc_commit(tmem_full);
             if (!ok || *abort_flag) {
