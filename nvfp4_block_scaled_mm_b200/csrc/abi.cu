@@ -127,7 +127,8 @@ nvfp4lora_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
 // 2-D row-major tensor [rows, cols] of `esize`-byte elements, read in boxes of
 // box_cols x box_rows with the 128-byte swizzle; out-of-range elements read as zero.
 nvfp4lora_status encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int esize,
-                           uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+                           uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
     nvfp4lora_status st = get_encoder(&enc);
     if (st != NVFP4LORA_OK) return st;
@@ -136,7 +137,7 @@ nvfp4lora_status encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataTy
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(NVFP4LORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
     return NVFP4LORA_OK;
@@ -206,7 +207,7 @@ nvfp4lora_status check_base(const uint8_t* a, const uint8_t* b, const uint8_t* a
 // GEMM launch
 // ---------------------------------------------------------------------------------------
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 
 template <Mode MODE>
 nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
@@ -222,15 +223,22 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     constexpr int smem = GemmSmem<kStages>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
-    CUtensorMap tm_a, tm_b, tm_d, tm_lb;
+    CUtensorMap tm_a, tm_b, tm_d, tm_lb, tm_out;
     std::memset(&tm_d, 0, sizeof(tm_d));
     std::memset(&tm_lb, 0, sizeof(tm_lb));
+    std::memset(&tm_out, 0, sizeof(tm_out));
     if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, kTileM)) != NVFP4LORA_OK) return st;
     if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, kTileN)) != NVFP4LORA_OK) return st;
     if (MODE != Mode::Off) {
         if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, kTileM)) != NVFP4LORA_OK) return st;
         if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, kTileN)) != NVFP4LORA_OK) return st;
     }
+    // rows of out 16-byte aligned: the epilogue writes 32 x 32 bf16 boxes with TMA stores
+    const bool vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16)));
+    if (vec_out &&
+        (st = encode_2d(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, kOutBoxCols, kOutBoxRows,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4LORA_OK)
+        return st;
 
     GemmArgs args;
     args.a_sf = a_sf;
@@ -251,7 +259,7 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     args.k_stages = (int)(K / 256);
     args.sf_atoms_k = (int)(K / 64);
     args.sf_row_blocks_b = (int)((N + 127) / 128);
-    args.vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16))) ? 1 : 0;
+    args.vec_out = vec_out ? 1 : 0;
 
     const int grid = (int)std::min<int64_t>(tiles, info->sms);
     cudaLaunchConfig_t cfg = {};
@@ -264,7 +272,7 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, args);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_out, args);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
     return NVFP4LORA_OK;
 }

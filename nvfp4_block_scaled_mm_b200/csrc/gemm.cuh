@@ -6,19 +6,22 @@
 //   warp 0     TMA producer: A/B code tiles (2-D TMA, 128-byte swizzle) and the 512-byte scale
 //              atoms (1-D bulk copies) per 256-wide K stage; after a tile's base stages, the
 //              d / lora_b tiles of the LoRA term (64 ranks per stage).
-//   warp 1     allocates TMEM; one thread issues tcgen05.cp (scale atoms -> TMEM) and the
-//              block-scaled MMAs (kind::mxf4nvf4, 16-element UE4M3 scale vectors, M=128, N=256)
-//              into a 256-column fp32 accumulator, then the bf16 MMAs (kind::f16, K = r) of the
-//              LoRA term: on the prepared path into the accumulator after the base product
-//              ("Prepared path" bullet); on the raw path into a separate 128-column accumulator,
-//              one N-half at a time ("Raw path" bullet: alpha and lora_scale stay independent).
-//   warps 2-9  epilogue, two warps per TMEM lane quarter, each owning 128 of the 256 columns:
-//              tcgen05.ld of its half into registers, release of the accumulator (so the next
-//              tile's MMAs start), then v = alpha*acc [; v = fma(s, lora_acc, v)] [; v += bias],
-//              one round-to-nearest-even to bf16 and the stores.
+//   warp 1     allocates TMEM; one thread issues the block-scaled MMAs (kind::mxf4nvf4,
+//              16-element UE4M3 scale vectors, M=128, N=256) into a 256-column fp32
+//              accumulator, then the bf16 MMAs (kind::f16, K = r) of the LoRA term: on the
+//              prepared path into the accumulator after the base product ("Prepared path"
+//              bullet); on the raw path into a separate 128-column accumulator, one N-half at a
+//              time ("Raw path" bullet: alpha and lora_scale stay independent).
+//   warps 2-9  two warps per TMEM lane quarter.  Between epilogues they stage every K stage's
+//              scale atoms into a TMEM scale slot with tcgen05.st (the layout a
+//              32x128b.warpx4 copy of the atom gives), up to NSF stages ahead of the MMAs, so
+//              the MMA thread issues nothing but MMAs.  Once a tile's accumulator is complete
+//              each warp drains its 128 of the 256 columns with tcgen05.ld, releases the
+//              accumulator (so the next tile's MMAs start), then v = alpha*acc
+//              [; v = fma(s, lora_acc, v)] [; v += bias], one round-to-nearest-even to bf16 and
+//              the stores.
 // N = 256 per MMA instruction is what keeps the tensor pipe busy: a 128-wide instruction costs
-// nearly as long as a 256-wide one, and the per-stage scale copies are amortised over twice the
-// work.  Zero-adapter path (Parameters: lora_scale): every role reads the LoRA scalar; when it
+// nearly as long as a 256-wide one.  Zero-adapter path (Parameters: lora_scale): every role reads the LoRA scalar; when it
 // equals 0 no LoRA tile is loaded or multiplied and the epilogue is the adapter-off one, so the
 // output is bitwise the adapter-off output.
 #pragma once
@@ -49,8 +52,13 @@ struct GemmArgs {
 };
 
 constexpr int kTileM = 128;
+constexpr unsigned kStageBackoffNs = 100;   // staging/epilogue warps' sleep between empty polls
 constexpr int kTileN = 256;
 constexpr int kGemmThreads = 320;        // producer, MMA, 8 epilogue warps
+constexpr int kEpiWarps = 8;
+constexpr int kOutBoxCols = 32;          // TMA store box of the epilogue: 32 columns x 32 rows
+constexpr int kOutBoxRows = 32;
+constexpr int kOutBoxes = 3;             // per epilogue warp: a box is rewritten once its store has read it
 
 // Shared-memory plan of one CTA.  Each stage holds one A tile (128 rows x 128 bytes), one B
 // tile (256 rows x 128 bytes) and their scale atoms; a LoRA stage reuses the A/B slots for a
@@ -65,9 +73,17 @@ struct GemmSmem {
     static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
     static constexpr int SFA_OFF = B_OFF + STAGES * B_BYTES;
     static constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_BYTES;
-    static constexpr int BAR_OFF = SFB_OFF + STAGES * SFB_BYTES;
-    // full[S], empty[S], tmem_full, acc_empty, lacc_full, lacc_empty, drain
-    static constexpr int NUM_BARS = 2 * STAGES + 5;
+    // the tile's 256 bias values (bf16), double-buffered across tiles
+    static constexpr int BIAS_BYTES = kTileN * 2;
+    static constexpr int BIAS_OFF = SFB_OFF + STAGES * SFB_BYTES;
+    // per epilogue warp, kOutBoxes 32 x 32 bf16 output boxes for TMA stores, used round-robin
+    static constexpr int OUT_BOX_BYTES = kOutBoxCols * kOutBoxRows * 2;
+    static constexpr int OUT_OFF = BIAS_OFF + 2 * BIAS_BYTES;
+    static constexpr int BAR_OFF = OUT_OFF + kEpiWarps * kOutBoxes * OUT_BOX_BYTES;
+    static constexpr int MAX_SLOTS = 8;                  // TMEM scale slots (at most)
+    // full[S], sf_full[S], empty[S], sf_ready[8], slot_free[8], tmem_full, acc_empty, lacc_full,
+    // lacc_empty, drain, bias_full[2], bias_empty[2]
+    static constexpr int NUM_BARS = 3 * STAGES + 2 * MAX_SLOTS + 9;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int DYN_BYTES = TOTAL + 1024;    // slack to align the base to 1024 bytes
@@ -75,9 +91,8 @@ struct GemmSmem {
 };
 
 // TMEM plan (columns of 32-bit cells, 128 lanes): the 256-column accumulator, NSF scale slots
-// used round-robin by the pipeline stages, and the raw path's 128-column LoRA accumulator.
-// tcgen05.cp and tcgen05.mma issued by one thread execute in issue order, so a slot is never
-// rewritten before the MMAs that read it have consumed it.
+// used round-robin by the base K stages, and the raw path's 128-column LoRA accumulator.  A slot
+// is rewritten only after the commit that follows the MMAs of its previous stage (slot_free).
 template <Mode MODE>
 struct TmemPlan {
     static constexpr int ACC = 0;
@@ -85,7 +100,7 @@ struct TmemPlan {
     static constexpr int SFA_COLS = 4 * 4;                // 4 MMAs (K = 64 each) x 4 columns
     static constexpr int SFB_COLS = 4 * (kTileN / 32);    // 4 MMAs x 8 columns
     static constexpr int SLOT_COLS = SFA_COLS + SFB_COLS;
-    // more slots let a stage's scale copies run further ahead of the MMAs still reading older slots
+    // more slots let the staging run further ahead of the MMAs still reading older slots
     static constexpr int NSF = (MODE == Mode::Raw) ? 2 : 5;
     static constexpr int LACC = SF0 + NSF * SLOT_COLS;    // raw path: 352
     static constexpr int USED = (MODE == Mode::Raw) ? LACC + 128 : LACC;
@@ -102,9 +117,10 @@ template <int STAGES, Mode MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_lb,
-                  const GemmArgs args) {
+                  const __grid_constant__ CUtensorMap tm_out, const GemmArgs args) {
     using L = GemmSmem<STAGES>;
     using T = TmemPlan<MODE>;
+    static_assert(T::NSF <= L::MAX_SLOTS, "scale slots exceed the barrier plan");
     constexpr uint32_t IDESC_F4 = idesc_nvf4(kTileN);
     constexpr uint32_t IDESC_BF16_FULL = idesc_bf16(kTileN);
     constexpr uint32_t IDESC_BF16_HALF = idesc_bf16(kTileN / 2);
@@ -113,12 +129,17 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-    uint64_t* empty = full + STAGES;
-    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* sf_full = full + STAGES;            // a stage's scale atoms are in shared memory
+    uint64_t* empty = sf_full + STAGES;
+    uint64_t* sf_ready = empty + STAGES;          // a slot holds its stage's scales in TMEM
+    uint64_t* slot_free = sf_ready + L::MAX_SLOTS;  // the MMAs that read a slot have completed
+    uint64_t* tmem_full = slot_free + L::MAX_SLOTS;
     uint64_t* acc_empty = tmem_full + 1;
     uint64_t* lacc_full = acc_empty + 1;
     uint64_t* lacc_empty = lacc_full + 1;
     uint64_t* drain = lacc_empty + 1;
+    uint64_t* bias_full = drain + 1;              // [2]: a tile's bias values are in shared memory
+    uint64_t* bias_empty = bias_full + 2;         // [2]: ... and every epilogue thread has read them
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -129,15 +150,25 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     if (threadIdx.x == 0) {
         prefetch_tensor_map(&tm_a);
         prefetch_tensor_map(&tm_b);
+        if (args.vec_out) prefetch_tensor_map(&tm_out);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&sf_full[s], 1);
             mbar_init(&empty[s], 1);
+        }
+        for (int k = 0; k < T::NSF; ++k) {
+            mbar_init(&sf_ready[k], 8);                // the 8 staging warps
+            mbar_init(&slot_free[k], 1);
         }
         mbar_init(tmem_full, 1);
         mbar_init(acc_empty, 256);
         mbar_init(lacc_full, 1);
         mbar_init(lacc_empty, 128);
         mbar_init(drain, 1);
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(&bias_full[k], 1);
+            mbar_init(&bias_empty[k], 32 * kEpiWarps);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -173,12 +204,27 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 prefetch_tensor_map(&tm_lb);
             }
             int stage = 0;
-            uint32_t phase = 0, filled = 0, filled_parity = 0;
+            // sf_full completes only for base stages, so its phases are counted per slot (sf_par)
+            uint32_t phase = 0, filled = 0, filled_parity = 0, scaled = 0, sf_par = 0, scaled_parity = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+            const bool bias_smem = args.bias != nullptr && args.vec_out;
+            int tl = 0;                                // local tile counter
+            uint32_t bias_issued = 0, bias_par = 0;    // per buffer: issued, parity of its last phase
+            for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x, ++tl) {
                 const int m_blk = tile % args.m_tiles;
                 const int n_blk = tile / args.m_tiles;
                 const int items = args.k_stages + (sv != 0.0f ? lora_chunks_if_on : 0);
+                if (bias_smem) {
+                    // the tile's bias slice, once the epilogue of two tiles ago has read the buffer
+                    const int bb = tl & 1;
+                    if (!mbar_wait(&bias_empty[bb], ((tl >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    const int n0 = n_blk * kTileN;
+                    const uint32_t bytes = (uint32_t)min(kTileN, args.N - n0) * 2u;   // N % 8 == 0
+                    mbar_arrive_expect_tx(&bias_full[bb], bytes);
+                    bulk_load(smem + L::BIAS_OFF + bb * L::BIAS_BYTES, args.bias + n0, bytes, &bias_full[bb]);
+                    bias_issued |= 1u << bb;
+                    bias_par = (bias_par & ~(1u << bb)) | ((((uint32_t)tl >> 1) & 1u) << bb);
+                }
                 for (int it = 0; it < items; ++it) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* sa = smem + L::A_OFF + stage * L::A_BYTES;
@@ -191,25 +237,38 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     } else {
                         const int rb0 = n_blk * (kTileN / 128);
                         const int nsfb = (rb0 + 1 < args.sf_row_blocks_b) ? 2 : 1;
-                        mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES + 2048 + nsfb * 2048);
-                        tma_load_2d(sa, &tm_a, &full[stage], it * 128, m_blk * kTileM);
-                        tma_load_2d(sb, &tm_b, &full[stage], it * 128, n_blk * kTileN);
+                        // the small scale atoms first, on their own barrier: the staging warps
+                        // put them into TMEM while the code tiles are still in flight
+                        mbar_arrive_expect_tx(&sf_full[stage], 2048 + nsfb * 2048);
                         bulk_load(smem + L::SFA_OFF + stage * L::SFA_BYTES,
-                                  args.a_sf + ((size_t)m_blk * args.sf_atoms_k + it * 4) * 512, 2048, &full[stage]);
+                                  args.a_sf + ((size_t)m_blk * args.sf_atoms_k + it * 4) * 512, 2048, &sf_full[stage]);
                         uint8_t* sfb = smem + L::SFB_OFF + stage * L::SFB_BYTES;
                         for (int j = 0; j < nsfb; ++j)
                             bulk_load(sfb + j * 2048, args.b_sf + ((size_t)(rb0 + j) * args.sf_atoms_k + it * 4) * 512,
-                                      2048, &full[stage]);
+                                      2048, &sf_full[stage]);
+                        mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
+                        tma_load_2d(sa, &tm_a, &full[stage], it * 128, m_blk * kTileM);
+                        tma_load_2d(sb, &tm_b, &full[stage], it * 128, n_blk * kTileN);
                     }
                     filled |= 1u << stage;
                     filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
+                    scaled = (scaled & ~(1u << stage)) | ((it < args.k_stages ? 1u : 0u) << stage);
+                    if (it < args.k_stages) {
+                        scaled_parity = (scaled_parity & ~(1u << stage)) | (sf_par & (1u << stage));
+                        sf_par ^= 1u << stage;
+                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok || *abort_flag) {
                 // Let every copy already issued land before the CTA can exit.
+                for (int k = 0; k < 2; ++k)
+                    if ((bias_issued >> k) & 1u) mbar_wait(&bias_full[k], (bias_par >> k) & 1u, nullptr);
                 for (int s = 0; s < STAGES; ++s)
-                    if ((filled >> s) & 1u) mbar_wait(&full[s], (filled_parity >> s) & 1u, nullptr);
+                    if ((filled >> s) & 1u) {
+                        mbar_wait(&full[s], (filled_parity >> s) & 1u, nullptr);
+                        if ((scaled >> s) & 1u) mbar_wait(&sf_full[s], (scaled_parity >> s) & 1u, nullptr);
+                    }
             }
         }
     } else if (warp == 1) {
@@ -219,7 +278,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             float sv = 0.0f;
             if constexpr (MODE != Mode::Off) sv = *args.scale;
             int stage = 0, slot = 0;
-            uint32_t phase = 0, lacc_waits = 0;
+            uint32_t phase = 0, slot_use = 0, lacc_waits = 0;
             bool ok = true;
             int i = 0;   // local tile counter
             for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x, ++i) {
@@ -227,26 +286,20 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 tc_fence_after();
                 // base product: k_stages x 4 MMAs of 128 x 256 x 64
                 for (int it = 0; ok && it < args.k_stages; ++it) {
+                    if (!mbar_wait(&sf_ready[slot], slot_use & 1u, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + L::A_OFF + stage * L::A_BYTES);
                     const uint32_t b_addr = smem_u32(smem + L::B_OFF + stage * L::B_BYTES);
                     const uint32_t sfa_t = tmem + T::SF0 + slot * T::SLOT_COLS;
                     const uint32_t sfb_t = sfa_t + T::SFA_COLS;
-                    const uint32_t sfa_s = smem_u32(smem + L::SFA_OFF + stage * L::SFA_BYTES);
-                    const uint32_t sfb_s = smem_u32(smem + L::SFB_OFF + stage * L::SFB_BYTES);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tc_copy_scale_atom(sfa_t + 4 * j, sdesc_scale_atom(sfa_s + j * 512));
-                        tc_copy_scale_atom(sfb_t + 8 * j, sdesc_scale_atom(sfb_s + j * 512));
-                        tc_copy_scale_atom(sfb_t + 8 * j + 4, sdesc_scale_atom(sfb_s + 2048 + j * 512));
-                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         tc_mma_nvf4(tmem + T::ACC, sdesc_sw128(a_addr + j * 32), sdesc_sw128(b_addr + j * 32),
                                     IDESC_F4, sfa_t + 4 * j, sfb_t + 8 * j, (it > 0 || j > 0) ? 1u : 0u);
                     tc_commit(&empty[stage]);
-                    if (++slot == T::NSF) slot = 0;
+                    tc_commit(&slot_free[slot]);
+                    if (++slot == T::NSF) { slot = 0; ++slot_use; }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
@@ -313,78 +366,161 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         }
         __syncwarp();
     } else {
-        // ------------------------------- epilogue -----------------------------------
+        // ------------------------- scale staging + epilogue -------------------------
         const int q = warp & 3;                        // TMEM lane quarter of this warp
         const int h = (warp - 2) >> 2;                 // which 128 of the 256 columns
         const int rl = q * 32 + lane;                  // row within the tile
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        constexpr uint32_t kAll = 0xffffffffu;
         grid_dependency_wait();
         float lora_s = 0.0f;
         if constexpr (MODE != Mode::Off) lora_s = *args.scale;
         const bool lora_on = (MODE != Mode::Off) && lora_s != 0.0f;
         const float alpha = *args.alpha;
-        int i = 0;
-        for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++i) {
-            const int m_blk = tile % args.m_tiles;
-            const int n_blk = tile / args.m_tiles;
-            if (!mbar_wait(tmem_full, i & 1, abort_flag)) break;
-            tc_fence_after();
-            uint32_t raw[128];
+        // the ring carries, per tile, the base K stages and then (LoRA on) the LoRA chunks: the
+        // same sequence the producer and the MMA thread walk
+        const int items = args.k_stages + (lora_on ? lora_chunks_if_on : 0);
+        int st_tile = blockIdx.x, st_it = 0, st_stage = 0;
+        uint32_t sf_par = 0;                           // per ring slot: parity of its next sf_full phase
+        uint32_t g = 0;                                // base stages staged so far
+        int epi_tile = blockIdx.x, i = 0;              // next tile to drain, local tile counter
+        unsigned long long idle_since = 0;
+        int out_box = 0;                               // next output box buffer of this warp
+        while (st_tile < args.num_tiles || epi_tile < args.num_tiles) {
+            bool progressed = false;
+            // 1) stage the next base stage's scales once its atoms have landed and its slot's
+            //    previous MMAs have completed (h = 0: the A scales, h = 1: the B scales)
+            if (st_tile < args.num_tiles) {
+                if (st_it >= args.k_stages) {
+                    progressed = true;                 // a LoRA chunk: nothing to stage
+                } else {
+                    const uint32_t slot = g % T::NSF, use = g / T::NSF;
+                    const bool ready = __all_sync(kAll, (use == 0 || mbar_test(&slot_free[slot], (use - 1) & 1u)) &&
+                                                            mbar_test(&sf_full[st_stage], (sf_par >> st_stage) & 1u));
+                    if (ready) {
+                        const uint32_t col = tmem + lane_off + T::SF0 + slot * T::SLOT_COLS;
+                        if (h == 0) {
+                            const uint8_t* src = smem + L::SFA_OFF + st_stage * L::SFA_BYTES + lane * 16;
+                            uint32_t v[16];
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_load_32(tmem + lane_off + T::ACC + h * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
-            tmem_load_wait();
-            tc_fence_before();
-            mbar_arrive(acc_empty);                    // the next tile's MMAs may start
-            float v[128];
+                            for (int j = 0; j < 4; ++j) {
+                                const uint4 w = *reinterpret_cast<const uint4*>(src + j * 512);
+                                v[4 * j] = w.x; v[4 * j + 1] = w.y; v[4 * j + 2] = w.z; v[4 * j + 3] = w.w;
+                            }
+                            tmem_store_16(col, v);
+                        } else {
+                            // per K step j: 4 columns from row block rb0's atom, then 4 from rb0 + 1's
+                            const uint8_t* src = smem + L::SFB_OFF + st_stage * L::SFB_BYTES + lane * 16;
+                            uint32_t v[32];
 #pragma unroll
-            for (int k = 0; k < 128; ++k) v[k] = __fmul_rn(alpha, __uint_as_float(raw[k]));
-            if (MODE == Mode::Raw && lora_on) {
-                if (h == 1 && !mbar_wait(lacc_full, i & 1, abort_flag)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t lv[16];
-                    tmem_load_16(tmem + lane_off + T::LACC + c * 16, lv);
-                    tmem_load_wait();
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) v[c * 16 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 16 + k]);
+                            for (int j = 0; j < 4; ++j) {
+                                const uint4 w0 = *reinterpret_cast<const uint4*>(src + j * 512);
+                                const uint4 w1 = *reinterpret_cast<const uint4*>(src + 2048 + j * 512);
+                                v[8 * j] = w0.x; v[8 * j + 1] = w0.y; v[8 * j + 2] = w0.z; v[8 * j + 3] = w0.w;
+                                v[8 * j + 4] = w1.x; v[8 * j + 5] = w1.y; v[8 * j + 6] = w1.z; v[8 * j + 7] = w1.w;
+                            }
+                            tmem_store_32(col + T::SFA_COLS, v);
+                        }
+                        tmem_store_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sf_ready[slot]);
+                        sf_par ^= 1u << st_stage;
+                        ++g;
+                        progressed = true;
+                    }
                 }
-                tc_fence_before();
-                mbar_arrive(lacc_empty);
+                if (progressed) {
+                    if (++st_stage == STAGES) st_stage = 0;
+                    if (++st_it == items) { st_it = 0; st_tile += gridDim.x; }
+                }
             }
-            const int row = m_blk * kTileM + rl;
-            const int col0 = n_blk * kTileN + h * 128;
-            const bool vec = args.vec_out && (col0 + 128 <= args.N);
-            if (args.bias != nullptr) {
-                if (vec) {
-                    const uint4* bp = reinterpret_cast<const uint4*>(args.bias + col0);
+            // 2) drain the next tile once its accumulator is complete
+            if (!progressed && epi_tile < args.num_tiles && __all_sync(kAll, mbar_test(tmem_full, i & 1))) {
+                const int tile = epi_tile;
+                const int m_blk = tile % args.m_tiles;
+                const int n_blk = tile / args.m_tiles;
+                tc_fence_after();
+                uint32_t raw[128];
+    #pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    tmem_load_32(tmem + lane_off + T::ACC + h * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
+                tmem_load_wait();
+                tc_fence_before();
+                mbar_arrive(acc_empty);                    // the next tile's MMAs may start
+                float v[128];
+    #pragma unroll
+                for (int k = 0; k < 128; ++k) v[k] = __fmul_rn(alpha, __uint_as_float(raw[k]));
+                if (MODE == Mode::Raw && lora_on) {
+                    if (h == 1 && !mbar_wait(lacc_full, i & 1, abort_flag)) break;
+                    tc_fence_after();
+    #pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t lv[16];
+                        tmem_load_16(tmem + lane_off + T::LACC + c * 16, lv);
+                        tmem_load_wait();
+    #pragma unroll
+                        for (int k = 0; k < 16; ++k) v[c * 16 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 16 + k]);
+                    }
+                    tc_fence_before();
+                    mbar_arrive(lacc_empty);
+                }
+                const int row = m_blk * kTileM + rl;
+                const int col0 = n_blk * kTileN + h * 128;
+                if (args.bias != nullptr) {
+                    if (args.vec_out) {
+                        // the producer put the tile's bias slice in shared memory (past N the
+                        // values are stale, and those columns are clipped by the TMA store)
+                        if (!mbar_wait(&bias_full[i & 1], (i >> 1) & 1, abort_flag)) break;
+                        const uint4* bp =
+                            reinterpret_cast<const uint4*>(smem + L::BIAS_OFF + (i & 1) * L::BIAS_BYTES) + h * 16;
 #pragma unroll
-                    for (int g = 0; g < 16; ++g) {
-                        const uint4 w = __ldg(bp + g);
-                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                        for (int g8 = 0; g8 < 16; ++g8) {
+                            const uint4 w = bp[g8];
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            v[g * 8 + 2 * e] = __fadd_rn(v[g * 8 + 2 * e], __uint_as_float(ws[e] << 16));
-                            v[g * 8 + 2 * e + 1] = __fadd_rn(v[g * 8 + 2 * e + 1], __uint_as_float(ws[e] & 0xFFFF0000u));
+                            for (int e = 0; e < 4; ++e) {
+                                v[g8 * 8 + 2 * e] = __fadd_rn(v[g8 * 8 + 2 * e], __uint_as_float(ws[e] << 16));
+                                v[g8 * 8 + 2 * e + 1] = __fadd_rn(v[g8 * 8 + 2 * e + 1], __uint_as_float(ws[e] & 0xFFFF0000u));
+                            }
+                        }
+                        mbar_arrive(&bias_empty[i & 1]);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 128; ++k)
+                            if (col0 + k < args.N)
+                                v[k] = __fadd_rn(v[k], __uint_as_float((uint32_t)__ldg(args.bias + col0 + k) << 16));
+                    }
+                }
+                if (args.vec_out) {
+                    // four 32 x 32 boxes per warp through kOutBoxes shared-memory buffers, each
+                    // written by a TMA store (rows past M and columns past N are clipped)
+                    uint8_t* box0 = smem + L::OUT_OFF + (warp - 2) * kOutBoxes * L::OUT_BOX_BYTES;
+                    const int y0 = m_blk * kTileM + q * 32;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint8_t* box = box0 + out_box * L::OUT_BOX_BYTES;
+                        if (++out_box == kOutBoxes) out_box = 0;
+                        // the buffer's previous store (kOutBoxes stores back) has read it
+                        if (lane == 0) bulk_wait_group_read<kOutBoxes - 1>();
+                        __syncwarp();
+                        uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int b8 = c * 32 + k * 8;
+                            dst[k] = make_uint4(pack_bf16x2(v[b8], v[b8 + 1]), pack_bf16x2(v[b8 + 2], v[b8 + 3]),
+                                                pack_bf16x2(v[b8 + 4], v[b8 + 5]), pack_bf16x2(v[b8 + 6], v[b8 + 7]));
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        const int x = col0 + c * kOutBoxCols;
+                        if (lane == 0 && x < args.N && y0 < args.M) {
+                            tma_store_2d(&tm_out, box, x, y0);
+                            bulk_commit_group();
                         }
                     }
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 128; ++k)
-                        if (col0 + k < args.N)
-                            v[k] = __fadd_rn(v[k], __uint_as_float((uint32_t)__ldg(args.bias + col0 + k) << 16));
-                }
-            }
-            if (row < args.M) {
-                uint16_t* orow = args.out + (size_t)row * args.N + col0;
-                if (vec) {
-                    uint4* op = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-                    for (int g = 0; g < 16; ++g)
-                        op[g] = make_uint4(pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]), pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]),
-                                           pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]), pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]));
-                } else {
+                } else if (row < args.M) {
+                    uint16_t* orow = args.out + (size_t)row * args.N + col0;
 #pragma unroll
                     for (int k = 0; k < 128; ++k)
                         if (col0 + k < args.N) {
@@ -392,8 +528,31 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                             orow[k] = *reinterpret_cast<uint16_t*>(&hv);
                         }
                 }
+                epi_tile += gridDim.x;
+                ++i;
+                progressed = true;
+            }
+            if (progressed) {
+                idle_since = 0;
+                continue;
+            }
+            if (__any_sync(kAll, *abort_flag != 0)) break;
+            // nothing ready: back off briefly, leaving the issue slots to the MMA and TMA threads
+            __nanosleep(kStageBackoffNs);
+            // bounded: give up (and tell the other roles) after kWaitLimitNs without progress
+            const unsigned long long now = global_timer_ns();
+            if (idle_since == 0) {
+                idle_since = now;
+            } else if (__shfl_sync(kAll, (now - idle_since > kWaitLimitNs) ? 1 : 0, 0)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicExch(&g_device_error, kErrTimeout);
+                }
+                break;
             }
         }
+        // the TMA stores have finished reading shared memory and writing out before the CTA ends
+        if (args.vec_out && lane == 0) bulk_wait_group_all();
     }
 
     tc_fence_before();
