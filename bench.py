@@ -40,13 +40,42 @@ WORKLOADS = {
     "cfg1": dict(src="cfg1", steps=20000),
     "cfg2": dict(src="cfg2", steps=2000),
     "cfg3": dict(src="cfg3", steps=100),
+    "cfg4": dict(src=None, steps=None),   # adapter-switch sweep (its own runner)
 }
 
 
 def describe(name):
-    from workloads import CONFIGS
+    from workloads import CFG4, CONFIGS
+    if name == "cfg4":
+        # the sweep's headline point (the reference arm times the oracle on it)
+        return dict(M=CFG4["Ms"][0], N=CFG4["N"], K=CFG4["K"], r=CFG4["rs"][0], path="raw",
+                    alpha=CFG4["alpha"], lora_scale=1.0, bias=False, seed=CFG4["seed"])
     c = dict(CONFIGS[WORKLOADS[name]["src"]])
     return c
+
+
+def time_graph(step, n, stream, device, warm=3):
+    """Capture n back-to-back calls of step(i) in one CUDA graph and time one replay with CUDA
+    events on the launching stream (after an untimed warm-up replay).  Returns ms per call."""
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            step(i)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step(i)
+    g.replay()
+    torch.cuda.synchronize(device)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        g.replay()
+        end.record(stream)
+    torch.cuda.synchronize(device)
+    ms = start.elapsed_time(end) / n
+    del g
+    return ms
 
 
 def algorithmic(c):
@@ -248,6 +277,25 @@ def run_ours(args, rank, world, device):
         ms = max_over_ranks(ms, device)
     ms_step = ms / K_steps
 
+    # LoRA overhead (outside the timed region): the same calls without an adapter, and on the
+    # prepared path the GEMM alone with the adapter already folded
+    n_extra = min(K_steps, 2000)
+
+    def step_off(i):
+        st = sets[i % copies]
+        L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, bias=st["bias"], out=out)
+
+    overhead = {"off_ms_per_call": time_graph(step_off, n_extra, stream, device)}
+    overhead["path_vs_off"] = ms_step / overhead["off_ms_per_call"] - 1.0
+    if prepared:
+        def step_gemm(i):
+            st = sets[i % copies]
+            L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, st["d"],
+                            lora_adapter=adapters[i % copies], bias=st["bias"], out=out)
+        overhead["gemm_ms_per_call"] = time_graph(step_gemm, n_extra, stream, device)
+        overhead["gemm_vs_off"] = overhead["gemm_ms_per_call"] / overhead["off_ms_per_call"] - 1.0
+    L.nvfp4lora_device_status(stream)
+
     # end to end through the public API with host buffers: per step, the activation-side
     # inputs (a, a_sf, d) go host -> device and the output comes back device -> host.
     e2e = run_e2e(L, p, sets[0], alpha, s, out, c, device, stream, min(K_steps, 2000), prepared,
@@ -255,7 +303,106 @@ def run_ours(args, rank, world, device):
 
     return dict(c=c, ms=ms, ms_step=ms_step, K=K_steps, W=max(W, 3), nbytes=nbytes, flops=flops,
                 lora_flops=lora_flops, copies=copies, clocks=clk.summary(), e2e=e2e,
-                launches=K_steps * launches_per_step, in_bytes=in_bytes, l2=l2, p=p)
+                launches=K_steps * launches_per_step, in_bytes=in_bytes, l2=l2, p=p, overhead=overhead)
+
+
+def cfg4_point(L, M, r, device, stream, l2):
+    """One point of the adapter-switch sweep: N=14336, K=4096, 8 adapters switched every call.
+    Times, each as a CUDA graph of back-to-back calls: the raw path with a different adapter's
+    pointers per call; the prepared path refolding the next adapter inside the graph (fold +
+    GEMM per call); and the prepared path with the next adapter's lora_b / lora_scale copied into
+    fixed captured sources before the refold."""
+    from workloads import CFG4, make_adapters, make_problem
+    N, K = CFG4["N"], CFG4["K"]
+    p = make_problem(M, N, K, r, CFG4["seed"] + 10 * M + r, alpha=CFG4["alpha"], lora_scale=1.0, bias=False)
+    w_bytes = p.b.numel() + p.b_sf.numel()
+    copies = max(1, math.ceil(3 * l2 / w_bytes))
+    weights = [(p.b.to(device), p.b_sf.to(device)) for _ in range(copies)]
+    a, a_sf, d = p.a.to(device), p.a_sf.to(device), p.d.to(device)
+    adps = [(lb.to(device), torch.tensor([sv], dtype=torch.float32, device=device))
+            for lb, sv in make_adapters(N, r, CFG4["adapters"], CFG4["seed"] + r)]
+    alpha = torch.tensor([CFG4["alpha"]], dtype=torch.float32, device=device)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    c = dict(M=M, N=N, K=K, r=r, bias=False)
+    nbytes, flops, _ = algorithmic(c)
+    est = max(nbytes / 3e12, flops / 2e15)
+    n = max(50, min(2000, int(0.03 / est)))
+    na = len(adps)
+
+    def step_raw(i):
+        b, b_sf = weights[i % copies]
+        lb, sv = adps[i % na]
+        L.mm_nvfp4_lora(a, b, a_sf, b_sf, alpha, d, lb, sv, out=out)
+
+    adp = L.prepare_nvfp4_lora_adapter(adps[0][0], adps[0][1], alpha)
+
+    def step_refold(i):
+        b, b_sf = weights[i % copies]
+        lb, sv = adps[i % na]
+        L.prepare_nvfp4_lora_adapter(lb, sv, alpha, out=adp)
+        L.mm_nvfp4_lora(a, b, a_sf, b_sf, alpha, d, lora_adapter=adp, out=out)
+
+    src_lb = adps[0][0].clone()
+    src_s = adps[0][1].clone()
+    adp2 = L.prepare_nvfp4_lora_adapter(src_lb, src_s, alpha)
+
+    def step_copy(i):
+        b, b_sf = weights[i % copies]
+        lb, sv = adps[i % na]
+        src_lb.copy_(lb)
+        src_s.copy_(sv)
+        L.prepare_nvfp4_lora_adapter(src_lb, src_s, alpha, out=adp2)
+        L.mm_nvfp4_lora(a, b, a_sf, b_sf, alpha, d, lora_adapter=adp2, out=out)
+
+    res = dict(M=M, r=r, calls=n, weight_copies=copies, algorithmic_bytes=nbytes, flops=flops)
+    for name, fn in (("raw_swap", step_raw), ("prepared_refold", step_refold), ("prepared_copy_refold", step_copy)):
+        ms = time_graph(fn, n, stream, device)
+        res[name] = {"us_per_call": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9, "tflops": flops / (ms * 1e-3) / 1e12}
+    L.nvfp4lora_device_status(stream)
+    return res
+
+
+def run_cfg4(args, rank, world, device):
+    """The adapter-switch sweep (M x r grid).  The line's value is the raw path's HBM throughput
+    at the decode point (M=1, r=8); every point is listed under "sweep"."""
+    import nvfp4_block_scaled_mm_b200 as L
+    from workloads import CFG4
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    stream = torch.cuda.Stream(device)
+    sweep = []
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        for M in CFG4["Ms"]:
+            for r in CFG4["rs"]:
+                sweep.append(cfg4_point(L, M, r, device, stream, l2))
+                torch.cuda.empty_cache()
+    head = sweep[0]
+    ms = head["raw_swap"]["us_per_call"] * 1e-3
+    if world > 1:
+        ms = max_over_ranks(ms, device)
+    value = head["algorithmic_bytes"] / (ms * 1e-3) / 1e9
+    peaks, peak_src = measured_peaks()
+    line = {
+        "metric": METRIC, "value": whole_job(value, world), "unit": "GB/s", "n_gpus": world, "steps": head["calls"],
+        "warmup": 3, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x ue4m3 -> fp32) + bf16 LoRA", "data": "synthetic",
+        "config": {"workload": f"cfg4: adapter-switch sweep N={CFG4['N']} K={CFG4['K']} M in {list(CFG4['Ms'])} "
+                               f"r in {list(CFG4['rs'])}, {CFG4['adapters']} adapters switched every call; "
+                               f"value = raw path at M=1 r=8",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2_defeat": "weights rotate through copies totalling >= 3x L2",
+                   "timing": "CUDA graph of back-to-back calls per point, CUDA events on the launching stream"},
+        "roofline": {"bound": "hbm", "achieved": value, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": value / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}", "traffic": None},
+        "clocks": clk.summary(),
+        "e2e": {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+                "note": "not measured for the sweep; the end-to-end figure is the cfg1 line's"},
+        # this library's kernels per call: raw 1; refold + GEMM 2 (the copy_ kernels are PyTorch's)
+        "gpu_launches": sum(pt["calls"] * k for pt in sweep for k in (1, 2, 2)),
+        "sweep": sweep,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
@@ -436,6 +583,11 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", device_id=device,
                                              timeout=datetime.timedelta(seconds=120))
+    if args.workload == "cfg4":
+        rc = run_cfg4(args, rank, world, device)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return rc
     res = run_ours(args, rank, world, device)
     c = res["c"]
     value, unit = metric_value(c, res["nbytes"], res["flops"], res["ms_step"])
@@ -465,6 +617,7 @@ def main():
         "gpu_launches": res["launches"],
         "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
         "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],
+        "lora_overhead": res["overhead"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(res["p"], c, res["nbytes"], res["flops"])
