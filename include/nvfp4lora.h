@@ -170,6 +170,17 @@ NVFP4LORA_API nvfp4lora_status nvfp4lora_mm_prepared(
  */
 NVFP4LORA_API nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream);
 
+/*
+ * Self-test of the failure path of the bounded waits (the pages have no counterpart; it lets a
+ * test exercise the path without faulting the GPU).  Enqueues on `stream` one CTA that waits
+ * on an mbarrier nothing completes, with the same wait helper as the GEMM kernels and a limit
+ * of limit_ns nanoseconds (0 < limit_ns <= 1e9) instead of 2 s.  The wait runs out and raises
+ * the device error word; the kernel then returns, so the context stays usable.  The next
+ * nvfp4lora_device_status returns NVFP4LORA_ERR_DEVICE_TIMEOUT and clears the word.
+ * Returns NVFP4LORA_ERR_INVALID_ARG (nothing enqueued) for a limit out of range.
+ */
+NVFP4LORA_API nvfp4lora_status nvfp4lora_selftest_wait_timeout(int64_t limit_ns, nvfp4lora_stream stream);
+
 /* Message of the last failing call on this host thread ("" when none). */
 NVFP4LORA_API const char* nvfp4lora_last_error(void);
 

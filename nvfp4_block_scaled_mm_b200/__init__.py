@@ -61,6 +61,8 @@ def _load():
     lib.nvfp4lora_mm_prepared.restype = ctypes.c_int
     lib.nvfp4lora_device_status.argtypes = [P]
     lib.nvfp4lora_device_status.restype = ctypes.c_int
+    lib.nvfp4lora_selftest_wait_timeout.argtypes = [I64, P]
+    lib.nvfp4lora_selftest_wait_timeout.restype = ctypes.c_int
     lib.nvfp4lora_last_error.argtypes = []
     lib.nvfp4lora_last_error.restype = ctypes.c_char_p
     lib.nvfp4lora_version.argtypes = []
@@ -168,6 +170,12 @@ def nvfp4lora_mm_prepared(a, b, a_sf, b_sf, alpha, d, adp, cur_lora_b, cur_lora_
 def nvfp4lora_device_status(stream=None) -> None:
     """Synchronise the stream and raise DeviceTimeoutError if a kernel's wait ran out."""
     _check(_lib.nvfp4lora_device_status(_stream(stream)))
+
+
+def nvfp4lora_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test: a wait that nothing completes runs out after
+    limit_ns; the next nvfp4lora_device_status raises DeviceTimeoutError."""
+    _check(_lib.nvfp4lora_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 # --------------------------------------------------------------------------------------

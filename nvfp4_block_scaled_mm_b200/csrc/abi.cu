@@ -25,6 +25,7 @@
 #include "gemm.cuh"
 #include "gemm_decode.cuh"
 #include "ptx.cuh"
+#include "selftest.cuh"
 
 namespace nvfp4lora {
 namespace {
@@ -558,6 +559,21 @@ nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream) {
         if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
         return fail(NVFP4LORA_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (pipeline stalled)");
     }
+    return NVFP4LORA_OK;
+}
+
+nvfp4lora_status nvfp4lora_selftest_wait_timeout(int64_t limit_ns, nvfp4lora_stream stream) {
+    t_last_error.clear();
+    if (limit_ns <= 0 || limit_ns > 1000000000)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "limit_ns = %lld: 0 < limit_ns <= 1e9 is required", (long long)limit_ns);
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+    wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)limit_ns);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
     return NVFP4LORA_OK;
 }
 

@@ -79,9 +79,10 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `parity` to complete.  Gives up when `*abort` (if given) becomes
-// non-zero, or after kWaitLimitNs; in the latter case it raises `*abort` and the device
-// error word.  Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// non-zero, or after `limit_ns` (default kWaitLimitNs); in the latter case it raises `*abort`
+// and the device error word.  Returns false when it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     while (true) {
@@ -89,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         for (int i = 0; i < 4; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (abort != nullptr && *abort) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             if (abort != nullptr) *abort = 1;
             atomicExch(&g_device_error, kErrTimeout);
             return false;

@@ -106,3 +106,13 @@ def test_prepare_rules(lib):
 def test_version_string(lib):
     lib.nvfp4lora_version.restype = ctypes.c_char_p
     assert b"sm_100a" in lib.nvfp4lora_version()
+
+
+def test_selftest_limit_is_checked_before_cuda(lib):
+    f = lib.nvfp4lora_selftest_wait_timeout
+    f.restype = ctypes.c_int
+    f.argtypes = [I64, P]
+    lib.nvfp4lora_last_error.restype = ctypes.c_char_p
+    for bad in (0, -5, 2_000_000_000):
+        assert f(bad, None) == 1
+        assert b"limit_ns" in lib.nvfp4lora_last_error()

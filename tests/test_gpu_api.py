@@ -154,3 +154,25 @@ def test_larger_scale_buffers_accepted(prob):
     got = L.mm_nvfp4_lora(x.a, x.b, big_a, big_b, x.alpha, x.d, x.lora_b, x.lora_scale, bias=x.bias)
     torch.cuda.synchronize()
     assert same(got, ref)
+
+
+def test_bounded_wait_runs_out_and_the_context_stays_usable(prob):
+    """The failure path of the kernels' bounded waits: a wait that nothing completes gives up
+    after its limit, the device error word reports it once, and the GPU keeps computing."""
+    import time
+    x = prob
+    L.nvfp4lora_device_status()                       # nothing pending
+    t0 = time.perf_counter()
+    L.nvfp4lora_selftest_wait_timeout(20_000_000)     # 20 ms
+    with pytest.raises(L.DeviceTimeoutError):
+        L.nvfp4lora_device_status()
+    waited = time.perf_counter() - t0
+    assert 0.015 < waited < 5.0, waited
+    L.nvfp4lora_device_status()                       # the word was cleared
+    # the context is intact: a GEMM after the timeout equals one before it, bit for bit
+    before = raw(x, x.d, x.lora_b, x.lora_scale)
+    torch.cuda.synchronize()
+    after = raw(x, x.d, x.lora_b, x.lora_scale)
+    torch.cuda.synchronize()
+    assert same(before, after)
+    L.nvfp4lora_device_status()
