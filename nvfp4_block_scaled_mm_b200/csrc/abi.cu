@@ -24,6 +24,7 @@
 #include "fold.cuh"
 #include "gemm.cuh"
 #include "gemm_decode.cuh"
+#include "gemm_pair.cuh"
 #include "ptx.cuh"
 #include "selftest.cuh"
 
@@ -374,13 +375,113 @@ nvfp4lora_status launch_decode(const uint8_t* a, const uint8_t* b, const uint8_t
     return launch_decode_mt<32, MODE>(info, a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
 }
 
-// Chooses the decode kernel for M <= 32 and the tiled kernel otherwise.
+// ---------------------------------------------------------------------------------------
+// SM-pair tiled launch (off / prepared, M > 128): clusters of 2 CTAs, 256 x 256 tiles
+// ---------------------------------------------------------------------------------------
+
+template <Mode MODE>
+nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                                  const float* alpha, const float* scale, const uint16_t* d, const uint16_t* lb,
+                                  int64_t r, const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                                  cudaStream_t stream) {
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+    auto kernel = nvfp4_gemm_pair_kernel<kPairStages, MODE>;
+    constexpr int smem = PairSmem<kPairStages>::DYN_BYTES;
+    if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
+
+    CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_d, tm_lb, tm_out;
+    std::memset(&tm_d, 0, sizeof(tm_d));
+    std::memset(&tm_lb, 0, sizeof(tm_lb));
+    std::memset(&tm_out, 0, sizeof(tm_out));
+    if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) != NVFP4LORA_OK) return st;
+    if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) != NVFP4LORA_OK) return st;
+    // the scale buffers as [bytes / 128, 128] (the 128x4 layout, rows padded to 128): a box of
+    // 16 rows is one 128-row block's 4 atoms of a K stage
+    const int64_t sfa_bytes = (M + 127) / 128 * 128 * (K / 16);
+    const int64_t sfb_bytes = (N + 127) / 128 * 128 * (K / 16);
+    if ((st = encode_2d(&tm_sfa, a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, sfa_bytes / 128, 128, 16,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4LORA_OK)
+        return st;
+    if ((st = encode_2d(&tm_sfb, b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, sfb_bytes / 128, 128, 16,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4LORA_OK)
+        return st;
+    if (MODE != Mode::Off) {
+        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, 128)) != NVFP4LORA_OK) return st;
+    }
+    const bool vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16)));
+    if (vec_out &&
+        (st = encode_2d(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, kOutBoxCols, kOutBoxRows,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4LORA_OK)
+        return st;
+
+    PairArgs args;
+    args.alpha = alpha;
+    args.scale = scale;
+    args.bias = bias;
+    args.out = out;
+    args.M = (int)M;
+    args.N = (int)N;
+    args.K = (int)K;
+    args.r = (int)r;
+    args.m_pairs = (int)((M + kPairTileM - 1) / kPairTileM);
+    args.n_tiles = (int)((N + kTileN - 1) / kTileN);
+    const int64_t tiles = (int64_t)args.m_pairs * args.n_tiles;
+    if (tiles > INT32_MAX) return fail(NVFP4LORA_ERR_INVALID_ARG, "too many output tiles (M x N too large)");
+    args.num_tiles = (int)tiles;
+    args.k_stages = (int)(K / 256);
+    args.sf_atoms_k = (int)(K / 64);
+    args.vec_out = vec_out ? 1 : 0;
+
+    const int pairs = (int)std::min<int64_t>(tiles, info->sms / 2);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_sfa, tm_sfb, tm_d, tm_lb, tm_out, args);
+    if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
+    return NVFP4LORA_OK;
+}
+
+// The SM-pair kernel measured level with the single-SM one where both run the same number of
+// waves, and worse where its 256-row tiles add a wave (or at M = 256): it is used from M = 512 on
+// when its wave count over the SM pairs is no larger than the single-SM kernel's over the SMs.
+bool use_pair_kernel(int64_t M, int64_t N) {
+    if (M < 512) return false;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    if (device_info(&dev, &info) != NVFP4LORA_OK) return false;
+    const int64_t n_tiles = (N + kTileN - 1) / kTileN;
+    const int64_t t1 = (M + kTileM - 1) / kTileM * n_tiles, t2 = (M + kPairTileM - 1) / kPairTileM * n_tiles;
+    const int64_t sms = info->sms, pairs = info->sms / 2;
+    return (t2 + pairs - 1) / pairs <= (t1 + sms - 1) / sms;
+}
+
+// Chooses the decode kernel for M <= 32, the SM-pair kernel for the off / prepared paths where
+// use_pair_kernel says so, and the single-SM tiled kernel otherwise.
 template <Mode MODE>
 nvfp4lora_status launch(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
                         const float* alpha, const float* scale, const uint16_t* d, const uint16_t* lb, int64_t r,
                         const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     if (M <= kDecodeMaxM)
         return launch_decode<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
+    if constexpr (MODE != Mode::Raw)
+        if (use_pair_kernel(M, N)) {
+            return launch_gemm_pair<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
+        }
     return launch_gemm<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
 }
 
