@@ -16,6 +16,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <string>
@@ -392,22 +393,26 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     constexpr int smem = PairSmem<kPairStages>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
-    CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb, tm_d, tm_lb, tm_out;
+    // The kernel splits its registers by warpgroup (setmaxnreg); the split assumes the launch's
+    // per-thread count that the compiler gave the kernel.  A different count would leave the
+    // epilogue warpgroups waiting for registers that never come, so refuse it here.
+    static std::atomic<int> checked{0};            // one per instantiation
+    if (!checked.load(std::memory_order_relaxed)) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+        if (e != cudaSuccess) return cuda_fail(e, "pair GEMM attributes");
+        if (fa.numRegs != kPairRegsLaunch)
+            return fail(NVFP4LORA_ERR_CUDA, "pair GEMM built with %d registers per thread, its register split assumes %d",
+                        fa.numRegs, kPairRegsLaunch);
+        checked.store(1, std::memory_order_relaxed);
+    }
+
+    CUtensorMap tm_a, tm_b, tm_d, tm_lb, tm_out;
     std::memset(&tm_d, 0, sizeof(tm_d));
     std::memset(&tm_lb, 0, sizeof(tm_lb));
     std::memset(&tm_out, 0, sizeof(tm_out));
     if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) != NVFP4LORA_OK) return st;
     if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) != NVFP4LORA_OK) return st;
-    // the scale buffers as [bytes / 128, 128] (the 128x4 layout, rows padded to 128): a box of
-    // 16 rows is one 128-row block's 4 atoms of a K stage
-    const int64_t sfa_bytes = (M + 127) / 128 * 128 * (K / 16);
-    const int64_t sfb_bytes = (N + 127) / 128 * 128 * (K / 16);
-    if ((st = encode_2d(&tm_sfa, a_sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, sfa_bytes / 128, 128, 16,
-                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4LORA_OK)
-        return st;
-    if ((st = encode_2d(&tm_sfb, b_sf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 128, sfb_bytes / 128, 128, 16,
-                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4LORA_OK)
-        return st;
     if (MODE != Mode::Off) {
         if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128)) != NVFP4LORA_OK) return st;
         if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, 128)) != NVFP4LORA_OK) return st;
@@ -421,6 +426,8 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     PairArgs args;
     args.alpha = alpha;
     args.scale = scale;
+    args.a_sf = a_sf;
+    args.b_sf = b_sf;
     args.bias = bias;
     args.out = out;
     args.M = (int)M;
@@ -434,12 +441,14 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     args.num_tiles = (int)tiles;
     args.k_stages = (int)(K / 256);
     args.sf_atoms_k = (int)(K / 64);
+    args.sf_row_blocks_a = (int)((M + 127) / 128);
+    args.sf_row_blocks_b = (int)((N + 127) / 128);
     args.vec_out = vec_out ? 1 : 0;
 
     const int pairs = (int)std::min<int64_t>(tiles, info->sms / 2);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(kPairThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -451,7 +460,7 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_sfa, tm_sfb, tm_d, tm_lb, tm_out, args);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_out, args);
     if (e != cudaSuccess) return cuda_fail(e, "pair GEMM launch");
     return NVFP4LORA_OK;
 }

@@ -5,18 +5,26 @@
 // accumulator after the base product, alpha is applied once).  A cluster of two CTAs computes
 // one 256 x 256 output tile per step with tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64):
 //   * each CTA loads its own 128 rows of A and its half of the tile's 256 B rows (the leader the
-//     first 128), at the same shared-memory offsets, plus its A scale atoms and the scale atoms
-//     of all 256 B rows; the loads are cta_group::2 TMA copies whose bytes complete on the
-//     leader's barrier, so each SM moves 38 KB per K stage instead of 54 KB for the same work;
-//   * the leader's single MMA thread copies both CTAs' scale atoms into their TMEM
-//     (tcgen05.cp.cta_group::2) and issues the MMAs and, on the prepared path, the bf16 LoRA MMAs
-//     (kind::f16, N = 256) for both; stage releases and the tile hand-off are multicast commits
-//     to both CTAs' barriers;
+//     first 128), at the same shared-memory offsets, with cta_group::2 TMA copies whose bytes
+//     complete on the leader's barrier, so each SM moves 32 KB of codes per K stage instead of
+//     48 KB for the same work;
+//   * a second producer thread per CTA bulk-copies its A scale atoms and the scale atoms of all
+//     256 B rows into a ring of its own, which the staging warps recycle as soon as they have
+//     read it, so the scales of a stage arrive several stages ahead of its MMAs;
+//   * four staging warps per CTA (one per TMEM lane quarter) write the stage's scale atoms from
+//     shared memory into a TMEM scale slot with tcgen05.st, in the layout a 32x128b.warpx4 copy
+//     gives, and report to the leader.  A scale copy (tcgen05.cp) shares the tensor pipe with
+//     the MMAs; a register store does not, so the MMAs run back to back;
+//   * the leader's single MMA thread issues the block-scaled MMAs and, on the prepared path, the
+//     bf16 LoRA MMAs (kind::f16, N = 256) for both CTAs; stage, slot and accumulator hand-offs
+//     are multicast commits to both CTAs' barriers;
 //   * each CTA drains its own 128 accumulator lanes (8 epilogue warps, 128 columns each), then
 //     v = alpha*acc [+ bias], one RNE to bf16, TMA stores; its threads release the accumulator
 //     on the leader's barrier (remote arrivals from the peer).
-// The raw path keeps the single-SM kernel: its LoRA term needs a separate accumulator whose
-// 128-column halves do not match the pair's split of N.  No multicast load is used.
+// Registers are split by warpgroup (setmaxnreg): producer/MMA and staging warps give theirs to
+// the epilogue warpgroups.  The raw path keeps the single-SM kernel: its LoRA term needs a
+// separate accumulator whose 128-column halves do not match the pair's split of N.  No multicast
+// load is used.
 #pragma once
 
 #include <cstdint>
@@ -30,16 +38,30 @@ namespace nvfp4lora {
 
 constexpr int kPairTileM = 256;          // output rows per pair tile (128 per CTA)
 constexpr int kPairStages = 4;
+constexpr int kPairSfStages = 4;         // scale-atom ring (own barriers, recycled by staging)
+constexpr int kPairThreads = 512;        // 4 warpgroups: producer/MMA, staging, 2 x epilogue
+// Registers per thread after the split.  The block is launched with 512 x 128; the split must not
+// exceed that pool (setmaxnreg.inc waits for registers that the other warpgroups give back).
+constexpr int kPairRegsLaunch = 128;
+constexpr int kPairRegsCtl = 80;         // warpgroup 0: producers, MMA issuer, one idle warp
+constexpr int kPairRegsStage = 72;       // warpgroup 1: scale staging
+constexpr int kPairRegsEpi = 176;        // warpgroups 2 and 3: epilogue
+static_assert(128 * (kPairRegsCtl + kPairRegsStage) + 256 * kPairRegsEpi <= kPairThreads * kPairRegsLaunch,
+              "pair register split exceeds the launch's register pool");
 
 struct PairArgs {
     const float* alpha;
     const float* scale;      // Prepared: the fold's ratio; Off: unused
+    const uint8_t* a_sf;     // 128x4-swizzled scale atoms of a
+    const uint8_t* b_sf;     // and of b
     const uint16_t* bias;    // bf16 [N] or null
     uint16_t* out;           // bf16 [M, N]
     int M, N, K, r;
     int m_pairs, n_tiles, num_tiles;   // pair tiles: m fastest
     int k_stages;            // K / 256
     int sf_atoms_k;          // K / 64
+    int sf_row_blocks_a;     // ceil(M / 128)
+    int sf_row_blocks_b;     // ceil(N / 128)
     int vec_out;             // rows of out (and bias) 16-byte aligned: TMA stores, bias in smem
 };
 
@@ -49,19 +71,21 @@ struct PairSmem {
     static constexpr int B_BYTES = 128 * 128;             // this CTA's half of the B tile
     static constexpr int SFA_BYTES = 4 * 512;             // 4 atoms: 128 rows x 4 K steps
     static constexpr int SFB_BYTES = 2 * 4 * 512;         // both 128-row blocks of the B tile
-    static constexpr int STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGE_TX = A_BYTES + B_BYTES;    // per CTA, on the leader's barrier
     static constexpr int LORA_TX = 128 * 128 + 128 * 128; // d rows + lora half, 64 ranks each
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
     static constexpr int SFA_OFF = B_OFF + STAGES * B_BYTES;
-    static constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_BYTES;
+    static constexpr int SFB_OFF = SFA_OFF + kPairSfStages * SFA_BYTES;
     static constexpr int BIAS_BYTES = kTileN * 2;
-    static constexpr int BIAS_OFF = SFB_OFF + STAGES * SFB_BYTES;
+    static constexpr int BIAS_OFF = SFB_OFF + kPairSfStages * SFB_BYTES;
     static constexpr int OUT_BOX_BYTES = kOutBoxCols * kOutBoxRows * 2;
     static constexpr int OUT_OFF = BIAS_OFF + 2 * BIAS_BYTES;
     static constexpr int BAR_OFF = OUT_OFF + kEpiWarps * kOutBoxes * OUT_BOX_BYTES;
-    // full[S], empty[S], tmem_full, acc_empty, drain, bias_full[2], bias_empty[2]
-    static constexpr int NUM_BARS = 2 * STAGES + 7;
+    static constexpr int MAX_SLOTS = 8;
+    // full[S], empty[S], sf_full[SF], sf_empty[SF], sf_ready[8], slot_free[8], tmem_full,
+    // acc_empty, drain, bias_full[2], bias_empty[2]
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * kPairSfStages + 2 * MAX_SLOTS + 7;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int DYN_BYTES = TOTAL + 1024;
@@ -69,8 +93,8 @@ struct PairSmem {
 };
 
 // TMEM (same columns in both CTAs): the 256-column accumulator and NSF scale slots, used round-
-// robin by the base stages.  Copies and MMAs come from one thread in issue order, so a slot is
-// rewritten only after the MMAs that read it.
+// robin by the base stages.  A slot is restaged only after the commit that follows the MMAs of
+// its previous stage (slot_free).
 struct PairTmem {
     static constexpr int ACC = 0;
     static constexpr int SF0 = kTileN;
@@ -80,12 +104,12 @@ struct PairTmem {
     static constexpr int NSF = 5;
     static constexpr int ALLOC = 512;
     static_assert(SF0 + NSF * SLOT_COLS <= ALLOC, "pair TMEM plan exceeds 512 columns");
+    static_assert(NSF <= PairSmem<kPairStages>::MAX_SLOTS, "too many scale slots for the barriers");
 };
 
 template <int STAGES, Mode MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
 nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                       const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                        const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_lb,
                        const __grid_constant__ CUtensorMap tm_out, const PairArgs args) {
     static_assert(MODE != Mode::Raw, "the raw path uses the single-SM kernel");
@@ -94,13 +118,18 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
     constexpr uint32_t IDESC_F4 = idesc_nvf4_m(kPairTileM, kTileN);
     constexpr uint32_t IDESC_BF16 = idesc_bf16_m(kPairTileM, kTileN);
     constexpr uint16_t kBoth = 0x3;
+    constexpr uint32_t kAll = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);   // the leader's is used
     uint64_t* empty = full + STAGES;
-    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* sf_full = empty + STAGES;            // this CTA's scale atoms are in shared memory
+    uint64_t* sf_empty = sf_full + kPairSfStages;  // its staging warps have read them
+    uint64_t* sf_ready = sf_empty + kPairSfStages; // the leader's: both CTAs staged a slot
+    uint64_t* slot_free = sf_ready + L::MAX_SLOTS; // the MMAs that read a slot have completed
+    uint64_t* tmem_full = slot_free + L::MAX_SLOTS;
     uint64_t* acc_empty = tmem_full + 1;                                // the leader's is used
     uint64_t* drain = acc_empty + 1;
     uint64_t* bias_full = drain + 1;
@@ -118,12 +147,18 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
     if (threadIdx.x == 0) {
         prefetch_tensor_map(&tm_a);
         prefetch_tensor_map(&tm_b);
-        prefetch_tensor_map(&tm_sfa);
-        prefetch_tensor_map(&tm_sfb);
         if (args.vec_out) prefetch_tensor_map(&tm_out);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);          // the leader's expect_tx; bytes from both CTAs
             mbar_init(&empty[s], 1);         // the leader's multicast commit
+        }
+        for (int s = 0; s < kPairSfStages; ++s) {
+            mbar_init(&sf_full[s], 1);       // this CTA's scale producer; its own bulk copies
+            mbar_init(&sf_empty[s], 4);      // this CTA's four staging warps
+        }
+        for (int k = 0; k < L::MAX_SLOTS; ++k) {
+            mbar_init(&sf_ready[k], 2 * 4);  // the four staging warps of each CTA
+            mbar_init(&slot_free[k], 1);     // the leader's multicast commit
         }
         mbar_init(tmem_full, 1);
         mbar_init(acc_empty, 2 * 32 * kEpiWarps);   // every epilogue thread of both CTAs
@@ -148,9 +183,11 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
     const uint32_t tmem = *tmem_slot;
     grid_launch_dependents();
 
-    if (warp == 0) {
-        // ------------------------------- TMA producer (both CTAs) -------------------------------
-        if (lane == 0) {
+    const int wg = warp >> 2;
+    if (wg == 0) {
+        reg_dealloc<kPairRegsCtl>();
+        if (warp == 0 && lane == 0) {
+            // ------------------------------- TMA producer (both CTAs) -------------------------------
             grid_dependency_wait();
             float sv = 0.0f;
             if constexpr (MODE == Mode::Prepared) sv = *args.scale;
@@ -161,14 +198,13 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             const bool lora_on = (MODE == Mode::Prepared) && sv != 0.0f;
             const bool bias_smem = args.bias != nullptr && args.vec_out;
             int stage = 0, tl = 0;
-            uint32_t phase = 0, filled = 0, bias_issued = 0, bias_par = 0;
+            uint32_t phase = 0, bias_issued = 0, bias_par = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < args.num_tiles; tile += npairs, ++tl) {
                 const int m_pair = tile % args.m_pairs;
                 const int n_blk = tile / args.m_pairs;
                 const int row_a = m_pair * kPairTileM + (int)rank * 128;      // this CTA's A rows
                 const int row_b = n_blk * kTileN + (int)rank * 128;           // this CTA's B half
-                const int blk_a = m_pair * 2 + (int)rank;                     // its 128-row scale block
                 if (bias_smem) {
                     const int bb = tl & 1;
                     if (!mbar_wait(&bias_empty[bb], ((tl >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -189,40 +225,67 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                         if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::STAGE_TX);
                         tma_load_2d_pair(sa, &tm_a, lead_full, it * 128, row_a);
                         tma_load_2d_pair(sb, &tm_b, lead_full, it * 128, row_b);
-                        // scale atoms through a [bytes / 128, 128] view: 16 rows = 4 atoms (2 KB)
-                        tma_load_2d_pair(smem + L::SFA_OFF + stage * L::SFA_BYTES, &tm_sfa, lead_full, 0,
-                                         (blk_a * args.sf_atoms_k + it * 4) * 4);
-                        uint8_t* sfb = smem + L::SFB_OFF + stage * L::SFB_BYTES;
-                        tma_load_2d_pair(sfb, &tm_sfb, lead_full, 0, ((n_blk * 2) * args.sf_atoms_k + it * 4) * 4);
-                        tma_load_2d_pair(sfb + 2048, &tm_sfb, lead_full, 0,
-                                         ((n_blk * 2 + 1) * args.sf_atoms_k + it * 4) * 4);
                     } else {
                         const int c = it - args.k_stages;
                         if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::LORA_TX);
                         tma_load_2d_pair(sa, &tm_d, lead_full, c * 64, row_a);
                         tma_load_2d_pair(sb, &tm_lb, lead_full, c * 64, row_b);
                     }
-                    filled |= 1u << stage;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok || *abort_flag) {
-                // Let this CTA's own copies land before it can exit (the pair's loads complete on
-                // the leader's barriers; both CTAs meet at the final cluster barrier).
+                // Let this CTA's own-barrier copies land before it can exit (the pair's code-tile
+                // loads complete on the leader's barriers; both CTAs meet at the final cluster
+                // barrier).
                 for (int k = 0; k < 2; ++k)
                     if ((bias_issued >> k) & 1u) mbar_wait(&bias_full[k], (bias_par >> k) & 1u, nullptr);
             }
-            (void)filled;
-        }
-    } else if (warp == 1) {
-        // ------------------------------- MMA issuer (the leader) -------------------------------
-        if (lane == 0 && rank == 0) {
+        } else if (warp == 2 && lane == 0) {
+            // ------------------------- scale-atom producer (both CTAs) -------------------------
+            // Per base K stage: this CTA's 4 A atoms (its 128-row block) and the 4 atoms of each of
+            // the tile's two 128-row B blocks, 512 bytes each, into the scale ring.  A block past the
+            // end of the scale buffer (rows past M or N only) is not copied: the TMEM columns it
+            // would fill scale only rows whose codes are zero-filled and whose outputs are clipped.
+            grid_dependency_wait();
+            int sst = 0;
+            uint32_t sphase = 0, issued = 0, issued_par = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < args.num_tiles; tile += npairs) {
+                const int m_pair = tile % args.m_pairs;
+                const int n_blk = tile / args.m_pairs;
+                const int blk_a = m_pair * 2 + (int)rank;
+                const bool has_a = blk_a < args.sf_row_blocks_a;
+                const int rb0 = n_blk * 2;
+                const int nsfb = (rb0 + 1 < args.sf_row_blocks_b) ? 2 : 1;
+                for (int it = 0; it < args.k_stages; ++it) {
+                    if (!mbar_wait(&sf_empty[sst], sphase ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&sf_full[sst], (has_a ? 2048u : 0u) + (uint32_t)nsfb * 2048u);
+                    if (has_a)
+                        bulk_load(smem + L::SFA_OFF + sst * L::SFA_BYTES,
+                                  args.a_sf + ((size_t)blk_a * args.sf_atoms_k + it * 4) * 512, 2048, &sf_full[sst]);
+                    uint8_t* sfb = smem + L::SFB_OFF + sst * L::SFB_BYTES;
+                    for (int j = 0; j < nsfb; ++j)
+                        bulk_load(sfb + j * 2048, args.b_sf + ((size_t)(rb0 + j) * args.sf_atoms_k + it * 4) * 512,
+                                  2048, &sf_full[sst]);
+                    issued |= 1u << sst;
+                    issued_par = (issued_par & ~(1u << sst)) | (sphase << sst);
+                    if (++sst == kPairSfStages) { sst = 0; sphase ^= 1; }
+                }
+            }
+            if (!ok || *abort_flag) {
+                // Let the copies already issued land before the CTA can exit.
+                for (int k = 0; k < kPairSfStages; ++k)
+                    if ((issued >> k) & 1u) mbar_wait(&sf_full[k], (issued_par >> k) & 1u, nullptr);
+            }
+        } else if (warp == 1 && lane == 0 && rank == 0) {
+            // ------------------------------- MMA issuer (the leader) -------------------------------
             grid_dependency_wait();
             float sv = 0.0f;
             if constexpr (MODE == Mode::Prepared) sv = *args.scale;
             const bool lora_on = (MODE == Mode::Prepared) && sv != 0.0f;
             int stage = 0, slot = 0;
-            uint32_t phase = 0;
+            uint32_t phase = 0, slot_use = 0;
             bool ok = true;
             int i = 0;
             for (int tile = pair; ok && tile < args.num_tiles; tile += npairs, ++i) {
@@ -230,26 +293,21 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                 if (!mbar_wait_cluster(acc_empty, (i & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int it = 0; ok && it < args.k_stages; ++it) {
+                    // both CTAs staged this slot's scales, and both CTAs' code tiles landed
+                    if (!mbar_wait_cluster(&sf_ready[slot], slot_use & 1u, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + L::A_OFF + stage * L::A_BYTES);
                     const uint32_t b_addr = smem_u32(smem + L::B_OFF + stage * L::B_BYTES);
                     const uint32_t sfa_t = tmem + T::SF0 + slot * T::SLOT_COLS;
                     const uint32_t sfb_t = sfa_t + T::SFA_COLS;
-                    const uint32_t sfa_s = smem_u32(smem + L::SFA_OFF + stage * L::SFA_BYTES);
-                    const uint32_t sfb_s = smem_u32(smem + L::SFB_OFF + stage * L::SFB_BYTES);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        tc_copy_scale_atom_pair(sfa_t + 4 * j, sdesc_scale_atom(sfa_s + j * 512));
-                        tc_copy_scale_atom_pair(sfb_t + 8 * j, sdesc_scale_atom(sfb_s + j * 512));
-                        tc_copy_scale_atom_pair(sfb_t + 8 * j + 4, sdesc_scale_atom(sfb_s + 2048 + j * 512));
-                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         tc_mma_nvf4_pair(tmem + T::ACC, sdesc_sw128(a_addr + j * 32), sdesc_sw128(b_addr + j * 32),
                                          IDESC_F4, sfa_t + 4 * j, sfb_t + 8 * j, (it > 0 || j > 0) ? 1u : 0u);
                     tc_commit_pair_multicast(&empty[stage], kBoth);
-                    if (++slot == T::NSF) slot = 0;
+                    tc_commit_pair_multicast(&slot_free[slot], kBoth);
+                    if (++slot == T::NSF) { slot = 0; ++slot_use; }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
@@ -279,10 +337,61 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             }
         }
         __syncwarp();
+    } else if (wg == 1) {
+        reg_dealloc<kPairRegsStage>();
+        // ------------------------------- scale staging (both CTAs) -------------------------------
+        // Per base K stage: this warp's TMEM lane quarter gets the 12 atoms' row `lane` (16 bytes
+        // each) as 4 columns per atom; the A atoms first (K steps 0..3), then per K step the two
+        // 128-row blocks of B.  Every lane quarter holds the whole atom, as a warpx4 copy leaves it.
+        const int q = warp & 3;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        grid_dependency_wait();
+        const uint32_t lead_sf_ready = map_to_rank(smem_u32(sf_ready), 0);
+        int sst = 0;
+        uint32_t sphase = 0, g = 0;
+        bool ok = true;
+        for (int tile = pair; ok && tile < args.num_tiles; tile += npairs) {
+            for (int it = 0; it < args.k_stages; ++it) {
+                const uint32_t slot = g % T::NSF, use = g / T::NSF;
+                if (!__all_sync(kAll, mbar_wait(&sf_full[sst], sphase, abort_flag))) { ok = false; break; }
+                const uint8_t* srca = smem + L::SFA_OFF + sst * L::SFA_BYTES + lane * 16;
+                const uint8_t* srcb = smem + L::SFB_OFF + sst * L::SFB_BYTES + lane * 16;
+                uint32_t va[16], vb[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(srca + j * 512);
+                    va[4 * j] = w.x; va[4 * j + 1] = w.y; va[4 * j + 2] = w.z; va[4 * j + 3] = w.w;
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(srcb + j * 512);
+                    const uint4 w1 = *reinterpret_cast<const uint4*>(srcb + 2048 + j * 512);
+                    vb[8 * j] = w0.x; vb[8 * j + 1] = w0.y; vb[8 * j + 2] = w0.z; vb[8 * j + 3] = w0.w;
+                    vb[8 * j + 4] = w1.x; vb[8 * j + 5] = w1.y; vb[8 * j + 6] = w1.z; vb[8 * j + 7] = w1.w;
+                }
+                // the slot's previous MMAs have completed (its loads overlap this wait)
+                if (use > 0 && !__all_sync(kAll, mbar_wait(&slot_free[slot], (use - 1) & 1u, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t col = tmem + lane_off + T::SF0 + slot * T::SLOT_COLS;
+                tmem_store_16(col, va);
+                tmem_store_32(col + T::SFA_COLS, vb);
+                // the stores have read their registers, so the loads are done: the ring slot is free
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_empty[sst]);
+                tmem_store_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(lead_sf_ready + slot * 8);
+                ++g;
+                if (++sst == kPairSfStages) { sst = 0; sphase ^= 1; }
+            }
+        }
     } else {
+        reg_alloc<kPairRegsEpi>();
         // ------------------------------- epilogue (both CTAs) -------------------------------
+        const int ew = warp - 8;                       // epilogue warp 0..7
         const int q = warp & 3;                        // TMEM lane quarter of this warp
-        const int h = (warp - 2) >> 2;                 // which 128 of the 256 columns
+        const int h = ew >> 2;                         // which 128 of the 256 columns
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         grid_dependency_wait();
         const float alpha = *args.alpha;
@@ -291,7 +400,7 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
         for (int tile = pair; tile < args.num_tiles; tile += npairs, ++i) {
             const int m_pair = tile % args.m_pairs;
             const int n_blk = tile / args.m_pairs;
-            if (!__all_sync(0xffffffffu, mbar_wait(tmem_full, i & 1, abort_flag))) break;
+            if (!__all_sync(kAll, mbar_wait(tmem_full, i & 1, abort_flag))) break;
             tc_fence_after();
             uint32_t raw[128];
 #pragma unroll
@@ -332,7 +441,7 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                 }
             }
             if (args.vec_out) {
-                uint8_t* box0 = smem + L::OUT_OFF + (warp - 2) * kOutBoxes * L::OUT_BOX_BYTES;
+                uint8_t* box0 = smem + L::OUT_OFF + ew * kOutBoxes * L::OUT_BOX_BYTES;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint8_t* box = box0 + out_box * L::OUT_BOX_BYTES;
