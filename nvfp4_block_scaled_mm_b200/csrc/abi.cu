@@ -212,6 +212,22 @@ nvfp4lora_status check_base(const uint8_t* a, const uint8_t* b, const uint8_t* a
 
 constexpr int kStages = 3;
 
+// The tiled kernels split their registers by warpgroup (setmaxnreg); the split assumes the per-
+// thread count the compiler gave the kernel at launch.  A smaller count would leave the epilogue
+// warpgroups waiting for registers that never come, so a build that differs is refused here.
+template <typename Kernel>
+nvfp4lora_status check_split_regs(Kernel kernel, int expected, std::atomic<int>& checked, const char* what) {
+    if (checked.load(std::memory_order_relaxed)) return NVFP4LORA_OK;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    if (fa.numRegs != expected)
+        return fail(NVFP4LORA_ERR_CUDA, "%s built with %d registers per thread, its register split assumes %d", what,
+                    fa.numRegs, expected);
+    checked.store(1, std::memory_order_relaxed);
+    return NVFP4LORA_OK;
+}
+
 template <Mode MODE>
 nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
                              const float* alpha, const float* scale, const uint16_t* d,
@@ -225,6 +241,8 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     auto kernel = nvfp4_gemm_kernel<kStages, MODE>;
     constexpr int smem = GemmSmem<kStages>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
+    static std::atomic<int> regs_ok{0};            // one per instantiation
+    if ((st = check_split_regs(kernel, kGemmRegsLaunch, regs_ok, "GEMM")) != NVFP4LORA_OK) return st;
 
     CUtensorMap tm_a, tm_b, tm_d, tm_lb, tm_out;
     std::memset(&tm_d, 0, sizeof(tm_d));
@@ -393,19 +411,8 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     constexpr int smem = PairSmem<kPairStages>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
 
-    // The kernel splits its registers by warpgroup (setmaxnreg); the split assumes the launch's
-    // per-thread count that the compiler gave the kernel.  A different count would leave the
-    // epilogue warpgroups waiting for registers that never come, so refuse it here.
-    static std::atomic<int> checked{0};            // one per instantiation
-    if (!checked.load(std::memory_order_relaxed)) {
-        cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
-        if (e != cudaSuccess) return cuda_fail(e, "pair GEMM attributes");
-        if (fa.numRegs != kPairRegsLaunch)
-            return fail(NVFP4LORA_ERR_CUDA, "pair GEMM built with %d registers per thread, its register split assumes %d",
-                        fa.numRegs, kPairRegsLaunch);
-        checked.store(1, std::memory_order_relaxed);
-    }
+    static std::atomic<int> regs_ok{0};            // one per instantiation
+    if ((st = check_split_regs(kernel, kPairRegsLaunch, regs_ok, "pair GEMM")) != NVFP4LORA_OK) return st;
 
     CUtensorMap tm_a, tm_b, tm_d, tm_lb, tm_out;
     std::memset(&tm_d, 0, sizeof(tm_d));

@@ -2,28 +2,31 @@
 //
 // Computes flashinfer.gemm.mm_nvfp4_lora's opening formula
 //     out = bf16_rne(alpha * (dequant(a) @ dequant(b)^T) + lora_scale * (d @ lora_b^T) [+ bias])
-// one 128 x 256 output tile at a time, tiles strided over a persistent grid:
-//   warp 0     TMA producer: A/B code tiles (2-D TMA, 128-byte swizzle) and the 512-byte scale
-//              atoms (1-D bulk copies) per 256-wide K stage; after a tile's base stages, the
-//              d / lora_b tiles of the LoRA term (64 ranks per stage).
-//   warp 1     allocates TMEM; one thread issues the block-scaled MMAs (kind::mxf4nvf4,
-//              16-element UE4M3 scale vectors, M=128, N=256) into a 256-column fp32
-//              accumulator, then the bf16 MMAs (kind::f16, K = r) of the LoRA term: on the
-//              prepared path into the accumulator after the base product ("Prepared path"
-//              bullet); on the raw path into a separate 128-column accumulator, one N-half at a
-//              time ("Raw path" bullet: alpha and lora_scale stay independent).
-//   warps 2-9  two warps per TMEM lane quarter.  Between epilogues they stage every K stage's
-//              scale atoms into a TMEM scale slot with tcgen05.st (the layout a
-//              32x128b.warpx4 copy of the atom gives), up to NSF stages ahead of the MMAs, so
-//              the MMA thread issues nothing but MMAs.  Once a tile's accumulator is complete
-//              each warp drains its 128 of the 256 columns with tcgen05.ld, releases the
-//              accumulator (so the next tile's MMAs start), then v = alpha*acc
-//              [; v = fma(s, lora_acc, v)] [; v += bias], one round-to-nearest-even to bf16 and
-//              the stores.
-// N = 256 per MMA instruction is what keeps the tensor pipe busy: a 128-wide instruction costs
-// nearly as long as a 256-wide one.  Zero-adapter path (Parameters: lora_scale): every role reads the LoRA scalar; when it
-// equals 0 no LoRA tile is loaded or multiplied and the epilogue is the adapter-off one, so the
-// output is bitwise the adapter-off output.
+// one 128 x 256 output tile at a time, tiles strided over a persistent grid.  Four warpgroups:
+//   warpgroup 0  warp 0: TMA producer of the A/B code tiles (2-D TMA, 128-byte swizzle) per
+//                256-wide K stage and, after a tile's base stages, of the d / lora_b tiles of
+//                the LoRA term (64 ranks per stage).  Warp 1: allocates TMEM; one thread issues
+//                the block-scaled MMAs (kind::mxf4nvf4, 16-element UE4M3 scale vectors, M=128,
+//                N=256) into a 256-column fp32 accumulator, then the bf16 MMAs (kind::f16,
+//                K = r) of the LoRA term: on the prepared path into the accumulator after the
+//                base product ("Prepared path" bullet); on the raw path into a separate 128-
+//                column accumulator, one N-half at a time ("Raw path" bullet: alpha and
+//                lora_scale stay independent).  Warp 2: bulk-copies each K stage's 512-byte
+//                scale atoms into a ring of its own.
+//   warpgroup 1  one warp per TMEM lane quarter: writes each stage's scale atoms from shared
+//                memory into a TMEM scale slot with tcgen05.st (the layout a 32x128b.warpx4
+//                copy of the atom gives), up to NSF stages ahead of the MMAs, so the MMA thread
+//                issues nothing but MMAs.  A tcgen05.cp scale copy would share the tensor pipe
+//                with the MMAs; a register store does not.
+//   warpgroups 2-3  two warps per TMEM lane quarter: once a tile's accumulator is complete each
+//                warp drains its 128 of the 256 columns with tcgen05.ld, releases the
+//                accumulator (so the next tile's MMAs start), then v = alpha*acc
+//                [; v = fma(s, lora_acc, v)] [; v += bias], one round-to-nearest-even to bf16 and
+//                TMA stores.
+// Registers are split by warpgroup (setmaxnreg).  N = 256 per MMA instruction halves the A-tile
+// traffic per flop against N = 128.  Zero-adapter path (Parameters: lora_scale): every role reads
+// the LoRA scalar; when it equals 0 no LoRA tile is loaded or multiplied and the epilogue is the
+// adapter-off one, so the output is bitwise the adapter-off output.
 #pragma once
 
 #include <cstdint>
@@ -52,17 +55,25 @@ struct GemmArgs {
 };
 
 constexpr int kTileM = 128;
-constexpr unsigned kStageBackoffNs = 100;   // staging/epilogue warps' sleep between empty polls
 constexpr int kTileN = 256;
-constexpr int kGemmThreads = 320;        // producer, MMA, 8 epilogue warps
 constexpr int kEpiWarps = 8;
 constexpr int kOutBoxCols = 32;          // TMA store box of the epilogue: 32 columns x 32 rows
 constexpr int kOutBoxRows = 32;
 constexpr int kOutBoxes = 3;             // per epilogue warp: a box is rewritten once its store has read it
+constexpr int kSfStages = 4;             // scale-atom ring (own barriers, recycled by the staging warps)
+constexpr int kGemmThreads = 512;        // 4 warpgroups: producers/MMA, staging, 2 x epilogue
+// Registers per thread after the split.  The block is launched with 512 x 128; the split must not
+// exceed that pool (setmaxnreg.inc waits for registers that the other warpgroups give back).
+constexpr int kGemmRegsLaunch = 128;
+constexpr int kGemmRegsCtl = 80;         // warpgroup 0: producers, MMA issuer, one idle warp
+constexpr int kGemmRegsStage = 72;       // warpgroup 1: scale staging
+constexpr int kGemmRegsEpi = 176;        // warpgroups 2 and 3: epilogue
+static_assert(128 * (kGemmRegsCtl + kGemmRegsStage) + 256 * kGemmRegsEpi <= kGemmThreads * kGemmRegsLaunch,
+              "register split exceeds the launch's register pool");
 
-// Shared-memory plan of one CTA.  Each stage holds one A tile (128 rows x 128 bytes), one B
-// tile (256 rows x 128 bytes) and their scale atoms; a LoRA stage reuses the A/B slots for a
-// 128 x 64 bf16 d tile and a 256 x 64 bf16 lora_b tile (also 128 bytes per row).
+// Shared-memory plan of one CTA.  Each stage holds one A tile (128 rows x 128 bytes) and one B
+// tile (256 rows x 128 bytes); a LoRA stage reuses them for a 128 x 64 bf16 d tile and a 256 x 64
+// bf16 lora_b tile (also 128 bytes per row).  The scale atoms of a stage sit in a ring of their own.
 template <int STAGES>
 struct GemmSmem {
     static constexpr int A_BYTES = kTileM * 128;
@@ -72,18 +83,18 @@ struct GemmSmem {
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
     static constexpr int SFA_OFF = B_OFF + STAGES * B_BYTES;
-    static constexpr int SFB_OFF = SFA_OFF + STAGES * SFA_BYTES;
+    static constexpr int SFB_OFF = SFA_OFF + kSfStages * SFA_BYTES;
     // the tile's 256 bias values (bf16), double-buffered across tiles
     static constexpr int BIAS_BYTES = kTileN * 2;
-    static constexpr int BIAS_OFF = SFB_OFF + STAGES * SFB_BYTES;
+    static constexpr int BIAS_OFF = SFB_OFF + kSfStages * SFB_BYTES;
     // per epilogue warp, kOutBoxes 32 x 32 bf16 output boxes for TMA stores, used round-robin
     static constexpr int OUT_BOX_BYTES = kOutBoxCols * kOutBoxRows * 2;
     static constexpr int OUT_OFF = BIAS_OFF + 2 * BIAS_BYTES;
     static constexpr int BAR_OFF = OUT_OFF + kEpiWarps * kOutBoxes * OUT_BOX_BYTES;
     static constexpr int MAX_SLOTS = 8;                  // TMEM scale slots (at most)
-    // full[S], sf_full[S], empty[S], sf_ready[8], slot_free[8], tmem_full, acc_empty, lacc_full,
-    // lacc_empty, drain, bias_full[2], bias_empty[2]
-    static constexpr int NUM_BARS = 3 * STAGES + 2 * MAX_SLOTS + 9;
+    // full[S], empty[S], sf_full[SF], sf_empty[SF], sf_ready[8], slot_free[8], tmem_full,
+    // acc_empty, lacc_full, lacc_empty, drain, bias_full[2], bias_empty[2]
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * kSfStages + 2 * MAX_SLOTS + 9;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int DYN_BYTES = TOTAL + 1024;    // slack to align the base to 1024 bytes
@@ -124,14 +135,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     constexpr uint32_t IDESC_F4 = idesc_nvf4(kTileN);
     constexpr uint32_t IDESC_BF16_FULL = idesc_bf16(kTileN);
     constexpr uint32_t IDESC_BF16_HALF = idesc_bf16(kTileN / 2);
+    constexpr uint32_t kAll = 0xffffffffu;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
-    uint64_t* sf_full = full + STAGES;            // a stage's scale atoms are in shared memory
-    uint64_t* empty = sf_full + STAGES;
-    uint64_t* sf_ready = empty + STAGES;          // a slot holds its stage's scales in TMEM
+    uint64_t* empty = full + STAGES;
+    uint64_t* sf_full = empty + STAGES;           // a stage's scale atoms are in shared memory
+    uint64_t* sf_empty = sf_full + kSfStages;     // ... and the staging warps have read them
+    uint64_t* sf_ready = sf_empty + kSfStages;    // a slot holds its stage's scales in TMEM
     uint64_t* slot_free = sf_ready + L::MAX_SLOTS;  // the MMAs that read a slot have completed
     uint64_t* tmem_full = slot_free + L::MAX_SLOTS;
     uint64_t* acc_empty = tmem_full + 1;
@@ -153,15 +166,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (args.vec_out) prefetch_tensor_map(&tm_out);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&sf_full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int s = 0; s < kSfStages; ++s) {
+            mbar_init(&sf_full[s], 1);
+            mbar_init(&sf_empty[s], 4);                // the 4 staging warps
+        }
         for (int k = 0; k < T::NSF; ++k) {
-            mbar_init(&sf_ready[k], 8);                // the 8 staging warps
+            mbar_init(&sf_ready[k], 4);                // the 4 staging warps
             mbar_init(&slot_free[k], 1);
         }
         mbar_init(tmem_full, 1);
-        mbar_init(acc_empty, 256);
+        mbar_init(acc_empty, 32 * kEpiWarps);
         mbar_init(lacc_full, 1);
         mbar_init(lacc_empty, 128);
         mbar_init(drain, 1);
@@ -184,9 +200,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     // now; every access to memory another kernel may write comes after grid_dependency_wait().
     grid_launch_dependents();
 
-    if (warp == 0) {
-        // ------------------------------- TMA producer -------------------------------
-        if (lane == 0) {
+    const int wg = warp >> 2;
+    if (wg == 0) {
+        reg_dealloc<kGemmRegsCtl>();
+        if (warp == 0 && lane == 0) {
+            // ------------------------------- TMA producer -------------------------------
             if (blockIdx.x < args.num_tiles) {
                 // warm L2 with the first stages of this CTA's first tile (a prefetch changes no
                 // data, so it may precede the dependency wait)
@@ -204,8 +222,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 prefetch_tensor_map(&tm_lb);
             }
             int stage = 0;
-            // sf_full completes only for base stages, so its phases are counted per slot (sf_par)
-            uint32_t phase = 0, filled = 0, filled_parity = 0, scaled = 0, sf_par = 0, scaled_parity = 0;
+            uint32_t phase = 0, filled = 0, filled_parity = 0;
             bool ok = true;
             const bool bias_smem = args.bias != nullptr && args.vec_out;
             int tl = 0;                                // local tile counter
@@ -229,34 +246,17 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* sa = smem + L::A_OFF + stage * L::A_BYTES;
                     uint8_t* sb = smem + L::B_OFF + stage * L::B_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
                     if (it >= args.k_stages) {
                         const int c = it - args.k_stages;
-                        mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
                         tma_load_2d(sa, &tm_d, &full[stage], c * 64, m_blk * kTileM);
                         tma_load_2d(sb, &tm_lb, &full[stage], c * 64, n_blk * kTileN);
                     } else {
-                        const int rb0 = n_blk * (kTileN / 128);
-                        const int nsfb = (rb0 + 1 < args.sf_row_blocks_b) ? 2 : 1;
-                        // the small scale atoms first, on their own barrier: the staging warps
-                        // put them into TMEM while the code tiles are still in flight
-                        mbar_arrive_expect_tx(&sf_full[stage], 2048 + nsfb * 2048);
-                        bulk_load(smem + L::SFA_OFF + stage * L::SFA_BYTES,
-                                  args.a_sf + ((size_t)m_blk * args.sf_atoms_k + it * 4) * 512, 2048, &sf_full[stage]);
-                        uint8_t* sfb = smem + L::SFB_OFF + stage * L::SFB_BYTES;
-                        for (int j = 0; j < nsfb; ++j)
-                            bulk_load(sfb + j * 2048, args.b_sf + ((size_t)(rb0 + j) * args.sf_atoms_k + it * 4) * 512,
-                                      2048, &sf_full[stage]);
-                        mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
                         tma_load_2d(sa, &tm_a, &full[stage], it * 128, m_blk * kTileM);
                         tma_load_2d(sb, &tm_b, &full[stage], it * 128, n_blk * kTileN);
                     }
                     filled |= 1u << stage;
                     filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
-                    scaled = (scaled & ~(1u << stage)) | ((it < args.k_stages ? 1u : 0u) << stage);
-                    if (it < args.k_stages) {
-                        scaled_parity = (scaled_parity & ~(1u << stage)) | (sf_par & (1u << stage));
-                        sf_par ^= 1u << stage;
-                    }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
@@ -265,15 +265,44 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 for (int k = 0; k < 2; ++k)
                     if ((bias_issued >> k) & 1u) mbar_wait(&bias_full[k], (bias_par >> k) & 1u, nullptr);
                 for (int s = 0; s < STAGES; ++s)
-                    if ((filled >> s) & 1u) {
-                        mbar_wait(&full[s], (filled_parity >> s) & 1u, nullptr);
-                        if ((scaled >> s) & 1u) mbar_wait(&sf_full[s], (scaled_parity >> s) & 1u, nullptr);
-                    }
+                    if ((filled >> s) & 1u) mbar_wait(&full[s], (filled_parity >> s) & 1u, nullptr);
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------- MMA issuer ---------------------------------
-        if (lane == 0) {
+        } else if (warp == 2 && lane == 0) {
+            // ------------------------------ scale-atom producer ------------------------------
+            // Per base K stage: the 4 A atoms of the tile's 128-row block and the 4 atoms of each
+            // of its two 128-row B blocks, 512 bytes each.  A B block past the end of b_sf (rows
+            // past N only) is not copied: the TMEM columns it would fill scale only rows whose
+            // codes are zero-filled and whose outputs are clipped.
+            grid_dependency_wait();
+            int sst = 0;
+            uint32_t sphase = 0, issued = 0, issued_par = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+                const int m_blk = tile % args.m_tiles;
+                const int n_blk = tile / args.m_tiles;
+                const int rb0 = n_blk * (kTileN / 128);
+                const int nsfb = (rb0 + 1 < args.sf_row_blocks_b) ? 2 : 1;
+                for (int it = 0; it < args.k_stages; ++it) {
+                    if (!mbar_wait(&sf_empty[sst], sphase ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&sf_full[sst], 2048u + (uint32_t)nsfb * 2048u);
+                    bulk_load(smem + L::SFA_OFF + sst * L::SFA_BYTES,
+                              args.a_sf + ((size_t)m_blk * args.sf_atoms_k + it * 4) * 512, 2048, &sf_full[sst]);
+                    uint8_t* sfb = smem + L::SFB_OFF + sst * L::SFB_BYTES;
+                    for (int j = 0; j < nsfb; ++j)
+                        bulk_load(sfb + j * 2048, args.b_sf + ((size_t)(rb0 + j) * args.sf_atoms_k + it * 4) * 512,
+                                  2048, &sf_full[sst]);
+                    issued |= 1u << sst;
+                    issued_par = (issued_par & ~(1u << sst)) | (sphase << sst);
+                    if (++sst == kSfStages) { sst = 0; sphase ^= 1; }
+                }
+            }
+            if (!ok || *abort_flag) {
+                // Let the copies already issued land before the CTA can exit.
+                for (int k = 0; k < kSfStages; ++k)
+                    if ((issued >> k) & 1u) mbar_wait(&sf_full[k], (issued_par >> k) & 1u, nullptr);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // ------------------------------- MMA issuer ---------------------------------
             grid_dependency_wait();
             float sv = 0.0f;
             if constexpr (MODE != Mode::Off) sv = *args.scale;
@@ -365,190 +394,161 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             }
         }
         __syncwarp();
+    } else if (wg == 1) {
+        reg_dealloc<kGemmRegsStage>();
+        // ------------------------------- scale staging -------------------------------
+        // Per base K stage: this warp's TMEM lane quarter gets the 12 atoms' row `lane` (16 bytes
+        // each) as 4 columns per atom; the A atoms first (K steps 0..3), then per K step the two
+        // 128-row blocks of B.  Every lane quarter holds the whole atom, as a warpx4 copy leaves it.
+        const int q = warp & 3;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        grid_dependency_wait();
+        int sst = 0;
+        uint32_t sphase = 0, g = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+            for (int it = 0; it < args.k_stages; ++it) {
+                const uint32_t slot = g % T::NSF, use = g / T::NSF;
+                if (!__all_sync(kAll, mbar_wait(&sf_full[sst], sphase, abort_flag))) { ok = false; break; }
+                const uint8_t* srca = smem + L::SFA_OFF + sst * L::SFA_BYTES + lane * 16;
+                const uint8_t* srcb = smem + L::SFB_OFF + sst * L::SFB_BYTES + lane * 16;
+                uint32_t va[16], vb[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(srca + j * 512);
+                    va[4 * j] = w.x; va[4 * j + 1] = w.y; va[4 * j + 2] = w.z; va[4 * j + 3] = w.w;
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(srcb + j * 512);
+                    const uint4 w1 = *reinterpret_cast<const uint4*>(srcb + 2048 + j * 512);
+                    vb[8 * j] = w0.x; vb[8 * j + 1] = w0.y; vb[8 * j + 2] = w0.z; vb[8 * j + 3] = w0.w;
+                    vb[8 * j + 4] = w1.x; vb[8 * j + 5] = w1.y; vb[8 * j + 6] = w1.z; vb[8 * j + 7] = w1.w;
+                }
+                // the slot's previous MMAs have completed (its loads overlap this wait)
+                if (use > 0 && !__all_sync(kAll, mbar_wait(&slot_free[slot], (use - 1) & 1u, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t col = tmem + lane_off + T::SF0 + slot * T::SLOT_COLS;
+                tmem_store_16(col, va);
+                tmem_store_32(col + T::SFA_COLS, vb);
+                // the stores have read their registers, so the loads are done: the ring slot is free
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_empty[sst]);
+                tmem_store_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[slot]);
+                ++g;
+                if (++sst == kSfStages) { sst = 0; sphase ^= 1; }
+            }
+        }
     } else {
-        // ------------------------- scale staging + epilogue -------------------------
+        reg_alloc<kGemmRegsEpi>();
+        // ------------------------------- epilogue -------------------------------
+        const int ew = warp - 8;                       // epilogue warp 0..7
         const int q = warp & 3;                        // TMEM lane quarter of this warp
-        const int h = (warp - 2) >> 2;                 // which 128 of the 256 columns
+        const int h = ew >> 2;                         // which 128 of the 256 columns
         const int rl = q * 32 + lane;                  // row within the tile
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        constexpr uint32_t kAll = 0xffffffffu;
         grid_dependency_wait();
         float lora_s = 0.0f;
         if constexpr (MODE != Mode::Off) lora_s = *args.scale;
         const bool lora_on = (MODE != Mode::Off) && lora_s != 0.0f;
         const float alpha = *args.alpha;
-        // the ring carries, per tile, the base K stages and then (LoRA on) the LoRA chunks: the
-        // same sequence the producer and the MMA thread walk
-        const int items = args.k_stages + (lora_on ? lora_chunks_if_on : 0);
-        int st_tile = blockIdx.x, st_it = 0, st_stage = 0;
-        uint32_t sf_par = 0;                           // per ring slot: parity of its next sf_full phase
-        uint32_t g = 0;                                // base stages staged so far
-        int epi_tile = blockIdx.x, i = 0;              // next tile to drain, local tile counter
-        unsigned long long idle_since = 0;
-        int out_box = 0;                               // next output box buffer of this warp
-        while (st_tile < args.num_tiles || epi_tile < args.num_tiles) {
-            bool progressed = false;
-            // 1) stage the next base stage's scales once its atoms have landed and its slot's
-            //    previous MMAs have completed (h = 0: the A scales, h = 1: the B scales)
-            if (st_tile < args.num_tiles) {
-                if (st_it >= args.k_stages) {
-                    progressed = true;                 // a LoRA chunk: nothing to stage
-                } else {
-                    const uint32_t slot = g % T::NSF, use = g / T::NSF;
-                    const bool ready = __all_sync(kAll, (use == 0 || mbar_test(&slot_free[slot], (use - 1) & 1u)) &&
-                                                            mbar_test(&sf_full[st_stage], (sf_par >> st_stage) & 1u));
-                    if (ready) {
-                        const uint32_t col = tmem + lane_off + T::SF0 + slot * T::SLOT_COLS;
-                        if (h == 0) {
-                            const uint8_t* src = smem + L::SFA_OFF + st_stage * L::SFA_BYTES + lane * 16;
-                            uint32_t v[16];
+        int i = 0, out_box = 0;
+        for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++i) {
+            const int m_blk = tile % args.m_tiles;
+            const int n_blk = tile / args.m_tiles;
+            if (!__all_sync(kAll, mbar_wait(tmem_full, i & 1, abort_flag))) break;
+            tc_fence_after();
+            uint32_t raw[128];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const uint4 w = *reinterpret_cast<const uint4*>(src + j * 512);
-                                v[4 * j] = w.x; v[4 * j + 1] = w.y; v[4 * j + 2] = w.z; v[4 * j + 3] = w.w;
-                            }
-                            tmem_store_16(col, v);
-                        } else {
-                            // per K step j: 4 columns from row block rb0's atom, then 4 from rb0 + 1's
-                            const uint8_t* src = smem + L::SFB_OFF + st_stage * L::SFB_BYTES + lane * 16;
-                            uint32_t v[32];
+            for (int c = 0; c < 4; ++c)
+                tmem_load_32(tmem + lane_off + T::ACC + h * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
+            tmem_load_wait();
+            tc_fence_before();
+            mbar_arrive(acc_empty);                    // the next tile's MMAs may start
+            float v[128];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const uint4 w0 = *reinterpret_cast<const uint4*>(src + j * 512);
-                                const uint4 w1 = *reinterpret_cast<const uint4*>(src + 2048 + j * 512);
-                                v[8 * j] = w0.x; v[8 * j + 1] = w0.y; v[8 * j + 2] = w0.z; v[8 * j + 3] = w0.w;
-                                v[8 * j + 4] = w1.x; v[8 * j + 5] = w1.y; v[8 * j + 6] = w1.z; v[8 * j + 7] = w1.w;
-                            }
-                            tmem_store_32(col + T::SFA_COLS, v);
-                        }
-                        tmem_store_wait();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sf_ready[slot]);
-                        sf_par ^= 1u << st_stage;
-                        ++g;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    if (++st_stage == STAGES) st_stage = 0;
-                    if (++st_it == items) { st_it = 0; st_tile += gridDim.x; }
-                }
-            }
-            // 2) drain the next tile once its accumulator is complete
-            if (!progressed && epi_tile < args.num_tiles && __all_sync(kAll, mbar_test(tmem_full, i & 1))) {
-                const int tile = epi_tile;
-                const int m_blk = tile % args.m_tiles;
-                const int n_blk = tile / args.m_tiles;
+            for (int k = 0; k < 128; ++k) v[k] = __fmul_rn(alpha, __uint_as_float(raw[k]));
+            if (MODE == Mode::Raw && lora_on) {
+                // half 0 of the LoRA accumulator is complete with the base one (tmem_full); half 1
+                // once lacc_full says so, after the h = 0 warps have released half 0
+                if (h == 1 && !__all_sync(kAll, mbar_wait(lacc_full, i & 1, abort_flag))) break;
                 tc_fence_after();
-                uint32_t raw[128];
-    #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tmem_load_32(tmem + lane_off + T::ACC + h * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(raw + c * 32));
-                tmem_load_wait();
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t lv[16];
+                    tmem_load_16(tmem + lane_off + T::LACC + c * 16, lv);
+                    tmem_load_wait();
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) v[c * 16 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 16 + k]);
+                }
                 tc_fence_before();
-                mbar_arrive(acc_empty);                    // the next tile's MMAs may start
-                float v[128];
-    #pragma unroll
-                for (int k = 0; k < 128; ++k) v[k] = __fmul_rn(alpha, __uint_as_float(raw[k]));
-                if (MODE == Mode::Raw && lora_on) {
-                    if (h == 1 && !mbar_wait(lacc_full, i & 1, abort_flag)) break;
-                    tc_fence_after();
-    #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        uint32_t lv[16];
-                        tmem_load_16(tmem + lane_off + T::LACC + c * 16, lv);
-                        tmem_load_wait();
-    #pragma unroll
-                        for (int k = 0; k < 16; ++k) v[c * 16 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 16 + k]);
-                    }
-                    tc_fence_before();
-                    mbar_arrive(lacc_empty);
-                }
-                const int row = m_blk * kTileM + rl;
-                const int col0 = n_blk * kTileN + h * 128;
-                if (args.bias != nullptr) {
-                    if (args.vec_out) {
-                        // the producer put the tile's bias slice in shared memory (past N the
-                        // values are stale, and those columns are clipped by the TMA store)
-                        if (!mbar_wait(&bias_full[i & 1], (i >> 1) & 1, abort_flag)) break;
-                        const uint4* bp =
-                            reinterpret_cast<const uint4*>(smem + L::BIAS_OFF + (i & 1) * L::BIAS_BYTES) + h * 16;
-#pragma unroll
-                        for (int g8 = 0; g8 < 16; ++g8) {
-                            const uint4 w = bp[g8];
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                v[g8 * 8 + 2 * e] = __fadd_rn(v[g8 * 8 + 2 * e], __uint_as_float(ws[e] << 16));
-                                v[g8 * 8 + 2 * e + 1] = __fadd_rn(v[g8 * 8 + 2 * e + 1], __uint_as_float(ws[e] & 0xFFFF0000u));
-                            }
-                        }
-                        mbar_arrive(&bias_empty[i & 1]);
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < 128; ++k)
-                            if (col0 + k < args.N)
-                                v[k] = __fadd_rn(v[k], __uint_as_float((uint32_t)__ldg(args.bias + col0 + k) << 16));
-                    }
-                }
+                mbar_arrive(lacc_empty);
+            }
+            const int row = m_blk * kTileM + rl;
+            const int col0 = n_blk * kTileN + h * 128;
+            if (args.bias != nullptr) {
                 if (args.vec_out) {
-                    // four 32 x 32 boxes per warp through kOutBoxes shared-memory buffers, each
-                    // written by a TMA store (rows past M and columns past N are clipped)
-                    uint8_t* box0 = smem + L::OUT_OFF + (warp - 2) * kOutBoxes * L::OUT_BOX_BYTES;
-                    const int y0 = m_blk * kTileM + q * 32;
+                    // the producer put the tile's bias slice in shared memory (past N the values
+                    // are stale, and those columns are clipped by the TMA store)
+                    if (!__all_sync(kAll, mbar_wait(&bias_full[i & 1], (i >> 1) & 1, abort_flag))) break;
+                    const uint4* bp =
+                        reinterpret_cast<const uint4*>(smem + L::BIAS_OFF + (i & 1) * L::BIAS_BYTES) + h * 16;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint8_t* box = box0 + out_box * L::OUT_BOX_BYTES;
-                        if (++out_box == kOutBoxes) out_box = 0;
-                        // the buffer's previous store (kOutBoxes stores back) has read it
-                        if (lane == 0) bulk_wait_group_read<kOutBoxes - 1>();
-                        __syncwarp();
-                        uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
+                    for (int g8 = 0; g8 < 16; ++g8) {
+                        const uint4 w = bp[g8];
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int b8 = c * 32 + k * 8;
-                            dst[k] = make_uint4(pack_bf16x2(v[b8], v[b8 + 1]), pack_bf16x2(v[b8 + 2], v[b8 + 3]),
-                                                pack_bf16x2(v[b8 + 4], v[b8 + 5]), pack_bf16x2(v[b8 + 6], v[b8 + 7]));
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        const int x = col0 + c * kOutBoxCols;
-                        if (lane == 0 && x < args.N && y0 < args.M) {
-                            tma_store_2d(&tm_out, box, x, y0);
-                            bulk_commit_group();
+                        for (int e = 0; e < 4; ++e) {
+                            v[g8 * 8 + 2 * e] = __fadd_rn(v[g8 * 8 + 2 * e], __uint_as_float(ws[e] << 16));
+                            v[g8 * 8 + 2 * e + 1] = __fadd_rn(v[g8 * 8 + 2 * e + 1], __uint_as_float(ws[e] & 0xFFFF0000u));
                         }
                     }
-                } else if (row < args.M) {
-                    uint16_t* orow = args.out + (size_t)row * args.N + col0;
+                    mbar_arrive(&bias_empty[i & 1]);
+                } else {
 #pragma unroll
                     for (int k = 0; k < 128; ++k)
-                        if (col0 + k < args.N) {
-                            __nv_bfloat16 hv = __float2bfloat16_rn(v[k]);
-                            orow[k] = *reinterpret_cast<uint16_t*>(&hv);
-                        }
+                        if (col0 + k < args.N)
+                            v[k] = __fadd_rn(v[k], __uint_as_float((uint32_t)__ldg(args.bias + col0 + k) << 16));
                 }
-                epi_tile += gridDim.x;
-                ++i;
-                progressed = true;
             }
-            if (progressed) {
-                idle_since = 0;
-                continue;
-            }
-            if (__any_sync(kAll, *abort_flag != 0)) break;
-            // nothing ready: back off briefly, leaving the issue slots to the MMA and TMA threads
-            __nanosleep(kStageBackoffNs);
-            // bounded: give up (and tell the other roles) after kWaitLimitNs without progress
-            const unsigned long long now = global_timer_ns();
-            if (idle_since == 0) {
-                idle_since = now;
-            } else if (__shfl_sync(kAll, (now - idle_since > kWaitLimitNs) ? 1 : 0, 0)) {
-                if (lane == 0) {
-                    *abort_flag = 1;
-                    atomicExch(&g_device_error, kErrTimeout);
+            if (args.vec_out) {
+                // four 32 x 32 boxes per warp through kOutBoxes shared-memory buffers, each
+                // written by a TMA store (rows past M and columns past N are clipped)
+                uint8_t* box0 = smem + L::OUT_OFF + ew * kOutBoxes * L::OUT_BOX_BYTES;
+                const int y0 = m_blk * kTileM + q * 32;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint8_t* box = box0 + out_box * L::OUT_BOX_BYTES;
+                    if (++out_box == kOutBoxes) out_box = 0;
+                    // the buffer's previous store (kOutBoxes stores back) has read it
+                    if (lane == 0) bulk_wait_group_read<kOutBoxes - 1>();
+                    __syncwarp();
+                    uint4* dst = reinterpret_cast<uint4*>(box + lane * 64);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int b8 = c * 32 + k * 8;
+                        dst[k] = make_uint4(pack_bf16x2(v[b8], v[b8 + 1]), pack_bf16x2(v[b8 + 2], v[b8 + 3]),
+                                            pack_bf16x2(v[b8 + 4], v[b8 + 5]), pack_bf16x2(v[b8 + 6], v[b8 + 7]));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    const int x = col0 + c * kOutBoxCols;
+                    if (lane == 0 && x < args.N && y0 < args.M) {
+                        tma_store_2d(&tm_out, box, x, y0);
+                        bulk_commit_group();
+                    }
                 }
-                break;
+            } else if (row < args.M) {
+                uint16_t* orow = args.out + (size_t)row * args.N + col0;
+#pragma unroll
+                for (int k = 0; k < 128; ++k)
+                    if (col0 + k < args.N) {
+                        __nv_bfloat16 hv = __float2bfloat16_rn(v[k]);
+                        orow[k] = *reinterpret_cast<uint16_t*>(&hv);
+                    }
             }
         }
         // the TMA stores have finished reading shared memory and writing out before the CTA ends
