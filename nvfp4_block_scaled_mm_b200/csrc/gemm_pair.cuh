@@ -409,8 +409,9 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             tmem_load_wait();
             tc_fence_before();
             // the leader may start the next tile's MMAs once both CTAs hold their accumulators
+            // (tcgen05.wait::ld has returned, so the arrival carries no data: relaxed suffices)
             if (rank == 0) mbar_arrive(acc_empty);
-            else mbar_arrive_remote(lead_acc_empty);
+            else mbar_arrive_remote_relaxed(lead_acc_empty);
             float v[128];
 #pragma unroll
             for (int k = 0; k < 128; ++k) v[k] = __fmul_rn(alpha, __uint_as_float(raw[k]));
