@@ -395,7 +395,7 @@ nvfp4lora_status launch_decode(const uint8_t* a, const uint8_t* b, const uint8_t
 }
 
 // ---------------------------------------------------------------------------------------
-// SM-pair tiled launch (off / prepared, M > 128): clusters of 2 CTAs, 256 x 256 tiles
+// SM-pair tiled launch: clusters of 2 CTAs, 256 x 256 tiles
 // ---------------------------------------------------------------------------------------
 
 template <Mode MODE>
@@ -422,7 +422,9 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) != NVFP4LORA_OK) return st;
     if (MODE != Mode::Off) {
         if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128)) != NVFP4LORA_OK) return st;
-        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, 128)) != NVFP4LORA_OK) return st;
+        // raw: per N-half, 64 of each CTA's 128 lora_b rows; prepared: all 128
+        const int lb_rows = (MODE == Mode::Raw) ? 64 : 128;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, lb_rows)) != NVFP4LORA_OK) return st;
     }
     const bool vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16)));
     if (vec_out &&
@@ -486,18 +488,16 @@ bool use_pair_kernel(int64_t M, int64_t N) {
     return (t2 + pairs - 1) / pairs <= (t1 + sms - 1) / sms;
 }
 
-// Chooses the decode kernel for M <= 32, the SM-pair kernel for the off / prepared paths where
-// use_pair_kernel says so, and the single-SM tiled kernel otherwise.
+// Chooses the decode kernel for M <= 32, the SM-pair kernel where use_pair_kernel says so, and the
+// single-SM tiled kernel otherwise.
 template <Mode MODE>
 nvfp4lora_status launch(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
                         const float* alpha, const float* scale, const uint16_t* d, const uint16_t* lb, int64_t r,
                         const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     if (M <= kDecodeMaxM)
         return launch_decode<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
-    if constexpr (MODE != Mode::Raw)
-        if (use_pair_kernel(M, N)) {
-            return launch_gemm_pair<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
-        }
+    if (use_pair_kernel(M, N))
+        return launch_gemm_pair<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
     return launch_gemm<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
 }
 

@@ -21,10 +21,12 @@
 //   * each CTA drains its own 128 accumulator lanes (8 epilogue warps, 128 columns each), then
 //     v = alpha*acc [+ bias], one RNE to bf16, TMA stores; its threads release the accumulator
 //     on the leader's barrier (remote arrivals from the peer).
+// Raw path ("Raw path" bullet: alpha and lora_scale stay independent): the LoRA term goes into a
+// separate 128-column accumulator, one N-half at a time (M = 256, N = 128 per instruction, each
+// CTA holding 64 of the half's lora_b rows); the epilogue warps of the first half read it and
+// release it before the second half is issued.
 // Registers are split by warpgroup (setmaxnreg): producer/MMA and staging warps give theirs to
-// the epilogue warpgroups.  The raw path keeps the single-SM kernel: its LoRA term needs a
-// separate accumulator whose 128-column halves do not match the pair's split of N.  No multicast
-// load is used.
+// the epilogue warpgroups.  No multicast load is used.
 #pragma once
 
 #include <cstdint>
@@ -84,26 +86,29 @@ struct PairSmem {
     static constexpr int BAR_OFF = OUT_OFF + kEpiWarps * kOutBoxes * OUT_BOX_BYTES;
     static constexpr int MAX_SLOTS = 8;
     // full[S], empty[S], sf_full[SF], sf_empty[SF], sf_ready[8], slot_free[8], tmem_full,
-    // acc_empty, drain, bias_full[2], bias_empty[2]
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * kPairSfStages + 2 * MAX_SLOTS + 7;
+    // acc_empty, lacc_full, lacc_empty, drain, bias_full[2], bias_empty[2]
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * kPairSfStages + 2 * MAX_SLOTS + 9;
     static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int DYN_BYTES = TOTAL + 1024;
     static_assert(DYN_BYTES <= 232448, "pair shared-memory plan exceeds 227 KB");
 };
 
-// TMEM (same columns in both CTAs): the 256-column accumulator and NSF scale slots, used round-
-// robin by the base stages.  A slot is restaged only after the commit that follows the MMAs of
-// its previous stage (slot_free).
+// TMEM (same columns in both CTAs): the 256-column accumulator, NSF scale slots used round-robin
+// by the base stages, and on the raw path the 128-column LoRA accumulator.  A slot is restaged
+// only after the commit that follows the MMAs of its previous stage (slot_free).
+template <Mode MODE>
 struct PairTmem {
     static constexpr int ACC = 0;
     static constexpr int SF0 = kTileN;
     static constexpr int SFA_COLS = 4 * 4;
     static constexpr int SFB_COLS = 4 * (kTileN / 32);
     static constexpr int SLOT_COLS = SFA_COLS + SFB_COLS;
-    static constexpr int NSF = 5;
+    static constexpr int NSF = (MODE == Mode::Raw) ? 2 : 5;
+    static constexpr int LACC = SF0 + NSF * SLOT_COLS;
+    static constexpr int USED = (MODE == Mode::Raw) ? LACC + 128 : LACC;
     static constexpr int ALLOC = 512;
-    static_assert(SF0 + NSF * SLOT_COLS <= ALLOC, "pair TMEM plan exceeds 512 columns");
+    static_assert(USED <= ALLOC, "pair TMEM plan exceeds 512 columns");
     static_assert(NSF <= PairSmem<kPairStages>::MAX_SLOTS, "too many scale slots for the barriers");
 };
 
@@ -112,11 +117,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                        const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_lb,
                        const __grid_constant__ CUtensorMap tm_out, const PairArgs args) {
-    static_assert(MODE != Mode::Raw, "the raw path uses the single-SM kernel");
     using L = PairSmem<STAGES>;
-    using T = PairTmem;
+    using T = PairTmem<MODE>;
     constexpr uint32_t IDESC_F4 = idesc_nvf4_m(kPairTileM, kTileN);
     constexpr uint32_t IDESC_BF16 = idesc_bf16_m(kPairTileM, kTileN);
+    constexpr uint32_t IDESC_BF16_HALF = idesc_bf16_m(kPairTileM, kTileN / 2);
     constexpr uint16_t kBoth = 0x3;
     constexpr uint32_t kAll = 0xffffffffu;
 
@@ -131,7 +136,9 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
     uint64_t* slot_free = sf_ready + L::MAX_SLOTS; // the MMAs that read a slot have completed
     uint64_t* tmem_full = slot_free + L::MAX_SLOTS;
     uint64_t* acc_empty = tmem_full + 1;                                // the leader's is used
-    uint64_t* drain = acc_empty + 1;
+    uint64_t* lacc_full = acc_empty + 1;           // raw: the second LoRA half is complete
+    uint64_t* lacc_empty = lacc_full + 1;          // raw, the leader's: a LoRA half has been read
+    uint64_t* drain = lacc_empty + 1;
     uint64_t* bias_full = drain + 1;
     uint64_t* bias_empty = bias_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
@@ -162,6 +169,8 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
         }
         mbar_init(tmem_full, 1);
         mbar_init(acc_empty, 2 * 32 * kEpiWarps);   // every epilogue thread of both CTAs
+        mbar_init(lacc_full, 1);
+        mbar_init(lacc_empty, 2 * 32 * (kEpiWarps / 2));   // one half's epilogue threads, both CTAs
         mbar_init(drain, 1);
         for (int k = 0; k < 2; ++k) {
             mbar_init(&bias_full[k], 1);
@@ -190,12 +199,12 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             // ------------------------------- TMA producer (both CTAs) -------------------------------
             grid_dependency_wait();
             float sv = 0.0f;
-            if constexpr (MODE == Mode::Prepared) sv = *args.scale;
-            if (MODE == Mode::Prepared) {
+            if constexpr (MODE != Mode::Off) sv = *args.scale;
+            if (MODE != Mode::Off) {
                 prefetch_tensor_map(&tm_d);
                 prefetch_tensor_map(&tm_lb);
             }
-            const bool lora_on = (MODE == Mode::Prepared) && sv != 0.0f;
+            const bool lora_on = (MODE != Mode::Off) && sv != 0.0f;
             const bool bias_smem = args.bias != nullptr && args.vec_out;
             int stage = 0, tl = 0;
             uint32_t phase = 0, bias_issued = 0, bias_par = 0;
@@ -229,7 +238,14 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                         const int c = it - args.k_stages;
                         if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::LORA_TX);
                         tma_load_2d_pair(sa, &tm_d, lead_full, c * 64, row_a);
-                        tma_load_2d_pair(sb, &tm_lb, lead_full, c * 64, row_b);
+                        if constexpr (MODE == Mode::Raw) {
+                            // per N-half, this CTA's 64 of its 128 lora_b rows (64-row boxes)
+                            const int r0 = n_blk * kTileN + (int)rank * 64;
+                            tma_load_2d_pair(sb, &tm_lb, lead_full, c * 64, r0);
+                            tma_load_2d_pair(sb + 64 * 128, &tm_lb, lead_full, c * 64, r0 + 128);
+                        } else {
+                            tma_load_2d_pair(sb, &tm_lb, lead_full, c * 64, row_b);
+                        }
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -282,17 +298,48 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             // ------------------------------- MMA issuer (the leader) -------------------------------
             grid_dependency_wait();
             float sv = 0.0f;
-            if constexpr (MODE == Mode::Prepared) sv = *args.scale;
-            const bool lora_on = (MODE == Mode::Prepared) && sv != 0.0f;
+            if constexpr (MODE != Mode::Off) sv = *args.scale;
+            const bool lora_on = (MODE != Mode::Off) && sv != 0.0f;
             int stage = 0, slot = 0;
-            uint32_t phase = 0, slot_use = 0;
+            uint32_t phase = 0, slot_use = 0, lacc_waits = 0;
             bool ok = true;
+            // Raw path: LoRA half `half` of a tile from its chunk stages s0 / s1 into the LoRA
+            // accumulator (M = 256, N = 128; each CTA holds 64 of the half's lora_b rows).
+            auto lora_half = [&](int half, int s0, int s1) {
+                for (int c = 0; c < lora_chunks_if_on; ++c) {
+                    const int stc = (c == 0) ? s0 : s1;
+                    const uint32_t a_addr = smem_u32(smem + L::A_OFF + stc * L::A_BYTES);
+                    const uint32_t b_addr = smem_u32(smem + L::B_OFF + stc * L::B_BYTES) + half * (64 * 128);
+                    const int rem = args.r - c * 64;
+                    const int ksteps = rem >= 64 ? 4 : (rem + 15) / 16;
+                    for (int j = 0; j < ksteps; ++j)
+                        tc_mma_bf16_pair(tmem + T::LACC, sdesc_sw128(a_addr + j * 32), sdesc_sw128(b_addr + j * 32),
+                                         IDESC_BF16_HALF, (c > 0 || j > 0) ? 1u : 0u);
+                }
+            };
+            // Raw path: the previous tile's LoRA half 1 waits until its half 0 has been read; it is
+            // issued a few stages into the next tile (or after its base stages, or at the end), so
+            // the tensor pipe does not idle meanwhile.  Its chunk stages stay held until then.
+            bool pend = false;
+            int pst0 = 0, pst1 = 0;
+            auto finish_pending = [&]() -> bool {
+                if (!mbar_wait_cluster(lacc_empty, (lacc_waits++ & 1) ^ 1, abort_flag)) return false;
+                tc_fence_after();
+                lora_half(1, pst0, pst1);
+                tc_commit_pair_multicast(lacc_full, kBoth);
+                tc_commit_pair_multicast(&empty[pst0], kBoth);
+                if (lora_chunks_if_on > 1) tc_commit_pair_multicast(&empty[pst1], kBoth);
+                pend = false;
+                return true;
+            };
+            constexpr int kDeferStages = 2;   // at most 2 of the 4 ring stages hold LoRA chunks
             int i = 0;
             for (int tile = pair; ok && tile < args.num_tiles; tile += npairs, ++i) {
                 // both CTAs' epilogues have read the previous tile's accumulator
                 if (!mbar_wait_cluster(acc_empty, (i & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int it = 0; ok && it < args.k_stages; ++it) {
+                    if (MODE == Mode::Raw && pend && it == kDeferStages && !finish_pending()) { ok = false; break; }
                     // both CTAs staged this slot's scales, and both CTAs' code tiles landed
                     if (!mbar_wait_cluster(&sf_ready[slot], slot_use & 1u, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
@@ -311,7 +358,7 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                if (lora_on) {
+                if (lora_on && MODE == Mode::Prepared) {
                     // the folded LoRA term into the same accumulator, after the base product
                     for (int c = 0; ok && c < lora_chunks_if_on; ++c) {
                         if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
@@ -327,9 +374,30 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                         if (++stage == STAGES) { stage = 0; phase ^= 1; }
                     }
                     if (!ok) break;
+                    tc_commit_pair_multicast(tmem_full, kBoth);   // both CTAs' accumulators are complete
+                } else if (lora_on && MODE == Mode::Raw) {
+                    // raw LoRA term in its own 128-column accumulator, one N-half at a time
+                    if (pend && !finish_pending()) { ok = false; break; }
+                    int st0 = 0, st1 = 0;      // stages of LoRA chunks 0 and 1 (r <= 128)
+                    for (int c = 0; ok && c < lora_chunks_if_on; ++c) {
+                        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                        if (c == 0) st0 = stage; else st1 = stage;
+                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    }
+                    // the previous tile's half 1 has been read
+                    if (ok && !mbar_wait_cluster(lacc_empty, (lacc_waits++ & 1) ^ 1, abort_flag)) ok = false;
+                    if (!ok) break;
+                    tc_fence_after();
+                    lora_half(0, st0, st1);
+                    tc_commit_pair_multicast(tmem_full, kBoth);   // base accumulator + LoRA half 0
+                    pend = true;
+                    pst0 = st0;
+                    pst1 = st1;
+                } else {
+                    tc_commit_pair_multicast(tmem_full, kBoth);   // both CTAs' accumulators are complete
                 }
-                tc_commit_pair_multicast(tmem_full, kBoth);     // both CTAs' accumulators are complete
             }
+            if (ok && MODE == Mode::Raw && pend && !finish_pending()) ok = false;
             if (!ok || *abort_flag) {
                 // Wait for the MMAs already issued before TMEM is released.
                 tc_commit_pair_multicast(drain, 0x1);
@@ -394,8 +462,12 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
         const int h = ew >> 2;                         // which 128 of the 256 columns
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         grid_dependency_wait();
+        float lora_s = 0.0f;
+        if constexpr (MODE == Mode::Raw) lora_s = *args.scale;
+        const bool raw_lora = (MODE == Mode::Raw) && lora_s != 0.0f;
         const float alpha = *args.alpha;
         const uint32_t lead_acc_empty = map_to_rank(smem_u32(acc_empty), 0);
+        const uint32_t lead_lacc_empty = map_to_rank(smem_u32(lacc_empty), 0);
         int i = 0, out_box = 0;
         for (int tile = pair; tile < args.num_tiles; tile += npairs, ++i) {
             const int m_pair = tile % args.m_pairs;
@@ -415,6 +487,23 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             float v[128];
 #pragma unroll
             for (int k = 0; k < 128; ++k) v[k] = __fmul_rn(alpha, __uint_as_float(raw[k]));
+            if (MODE == Mode::Raw && raw_lora) {
+                // half 0 of the LoRA accumulator is complete with the base one (tmem_full); half 1
+                // once lacc_full says so, after the h = 0 warps of both CTAs have released half 0
+                if (h == 1 && !__all_sync(kAll, mbar_wait(lacc_full, i & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t lv[16];
+                    tmem_load_16(tmem + lane_off + T::LACC + c * 16, lv);
+                    tmem_load_wait();
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) v[c * 16 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 16 + k]);
+                }
+                tc_fence_before();
+                if (rank == 0) mbar_arrive(lacc_empty);
+                else mbar_arrive_remote_relaxed(lead_lacc_empty);
+            }
             const int row0 = m_pair * kPairTileM + (int)rank * 128 + q * 32;   // this warp's 32 rows
             const int row = row0 + lane;
             const int col0 = n_blk * kTileN + h * 128;
