@@ -57,25 +57,39 @@ def describe(name):
 def time_graph(step, n, stream, device, warm=3):
     """Capture n back-to-back calls of step(i) in one CUDA graph and time one replay with CUDA
     events on the launching stream (after an untimed warm-up replay).  Returns ms per call."""
+    return time_graphs({"x": step}, n, stream, device, warm=warm, rounds=1)["x"]
+
+
+def time_graphs(steps, n, stream, device, warm=3, rounds=3):
+    """Like time_graph for several step functions at once: each is captured in its own graph of n
+    calls, and the graphs are replayed in turn `rounds` times, so clock and temperature drift falls
+    on all of them alike.  Returns the median ms per call of each."""
+    graphs = {}
     with torch.cuda.stream(stream):
-        for i in range(warm):
-            step(i)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
+        for name, step in steps.items():
+            for i in range(warm):
                 step(i)
-    g.replay()
-    torch.cuda.synchronize(device)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    step(i)
+            graphs[name] = g
+    for g in graphs.values():
         g.replay()
-        end.record(stream)
     torch.cuda.synchronize(device)
-    ms = start.elapsed_time(end) / n
-    del g
-    return ms
+    times = {name: [] for name in steps}
+    for _ in range(rounds):
+        for name, g in graphs.items():
+            start = torch.cuda.Event(enable_timing=True)
+            end = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                start.record(stream)
+                g.replay()
+                end.record(stream)
+            torch.cuda.synchronize(device)
+            times[name].append(start.elapsed_time(end) / n)
+    del graphs
+    return {name: sorted(v)[len(v) // 2] for name, v in times.items()}
 
 
 def algorithmic(c):
@@ -277,23 +291,29 @@ def run_ours(args, rank, world, device):
         ms = max_over_ranks(ms, device)
     ms_step = ms / K_steps
 
-    # LoRA overhead (outside the timed region): the same calls without an adapter, and on the
-    # prepared path the GEMM alone with the adapter already folded
+    # LoRA overhead (outside the timed region): the step, the same calls without an adapter, and
+    # on the prepared path the GEMM alone with the adapter already folded, timed in turn so that
+    # clock drift falls on all of them alike
     n_extra = min(K_steps, 2000)
 
     def step_off(i):
         st = sets[i % copies]
         L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, bias=st["bias"], out=out)
 
-    overhead = {"off_ms_per_call": time_graph(step_off, n_extra, stream, device)}
-    overhead["path_vs_off"] = ms_step / overhead["off_ms_per_call"] - 1.0
+    kinds = {"path": step, "off": step_off}
     if prepared:
         def step_gemm(i):
             st = sets[i % copies]
             L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, st["d"],
                             lora_adapter=adapters[i % copies], bias=st["bias"], out=out)
-        overhead["gemm_ms_per_call"] = time_graph(step_gemm, n_extra, stream, device)
-        overhead["gemm_vs_off"] = overhead["gemm_ms_per_call"] / overhead["off_ms_per_call"] - 1.0
+        kinds["gemm"] = step_gemm
+    t = time_graphs(kinds, n_extra, stream, device)
+    overhead = {"off_ms_per_call": t["off"], "path_ms_per_step": t["path"],
+                "path_vs_off": t["path"] / t["off"] - 1.0,
+                "method": "median of 3 interleaved replays of one graph of %d calls each" % n_extra}
+    if prepared:
+        overhead["gemm_ms_per_call"] = t["gemm"]
+        overhead["gemm_vs_off"] = t["gemm"] / t["off"] - 1.0
     L.nvfp4lora_device_status(stream)
 
     # end to end through the public API with host buffers: per step, the activation-side
