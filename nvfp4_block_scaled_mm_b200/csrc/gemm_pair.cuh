@@ -41,7 +41,10 @@ namespace nvfp4lora {
 constexpr int kPairTileM = 256;          // output rows per pair tile (128 per CTA)
 constexpr int kPairStages = 4;
 constexpr int kPairSfStages = 4;         // scale-atom ring (own barriers, recycled by staging)
-constexpr int kPairThreads = 512;        // 4 warpgroups: producer/MMA, staging, 2 x epilogue
+constexpr int kPairThreads = 512;
+// Raw path: a tile's second LoRA half is issued this many base stages into the next tile, so that
+// the epilogue warps have read the first half by then.
+constexpr int kRawHalf1At = 4;        // 4 warpgroups: producer/MMA, staging, 2 x epilogue
 // Registers per thread after the split.  The block is launched with 512 x 128; the split must not
 // exceed that pool (setmaxnreg.inc waits for registers that the other warpgroups give back).
 constexpr int kPairRegsLaunch = 128;
@@ -75,6 +78,7 @@ struct PairSmem {
     static constexpr int SFB_BYTES = 2 * 4 * 512;         // both 128-row blocks of the B tile
     static constexpr int STAGE_TX = A_BYTES + B_BYTES;    // per CTA, on the leader's barrier
     static constexpr int LORA_TX = 128 * 128 + 128 * 128; // d rows + lora half, 64 ranks each
+    static constexpr int LORA_HALF_TX = 128 * 128 + 64 * 128;  // raw: d rows + 64 lora rows of an N-half
     static constexpr int A_OFF = 0;
     static constexpr int B_OFF = A_OFF + STAGES * A_BYTES;
     static constexpr int SFA_OFF = B_OFF + STAGES * B_BYTES;
@@ -209,6 +213,40 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             int stage = 0, tl = 0;
             uint32_t phase = 0, bias_issued = 0, bias_par = 0;
             bool ok = true;
+            bool pend = false;                 // raw: the previous tile's LoRA half 1 is still due
+            int prev_m = 0, prev_n = 0;
+            // one ring item: wait for the stage, arm the leader's barrier, issue this CTA's loads
+            auto next_stage = [&](uint32_t tx, uint32_t& lead_full, uint8_t*& sa, uint8_t*& sb) -> bool {
+                if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) return false;
+                lead_full = map_to_rank(smem_u32(&full[stage]), 0);
+                sa = smem + L::A_OFF + stage * L::A_BYTES;
+                sb = smem + L::B_OFF + stage * L::B_BYTES;
+                if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * tx);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                return true;
+            };
+            auto emit_base = [&](int it, int row_a, int row_b) -> bool {
+                uint32_t lf; uint8_t *sa, *sb;
+                if (!next_stage(L::STAGE_TX, lf, sa, sb)) return false;
+                tma_load_2d_pair(sa, &tm_a, lf, it * 128, row_a);
+                tma_load_2d_pair(sb, &tm_b, lf, it * 128, row_b);
+                return true;
+            };
+            auto emit_lora = [&](int c, int row_a, int row_b) -> bool {   // prepared: d + lora_b rows
+                uint32_t lf; uint8_t *sa, *sb;
+                if (!next_stage(L::LORA_TX, lf, sa, sb)) return false;
+                tma_load_2d_pair(sa, &tm_d, lf, c * 64, row_a);
+                tma_load_2d_pair(sb, &tm_lb, lf, c * 64, row_b);
+                return true;
+            };
+            // raw: d rows + this CTA's 64 lora_b rows of N-half h (64-row boxes)
+            auto emit_half = [&](int c, int h, int m_pair, int n_blk) -> bool {
+                uint32_t lf; uint8_t *sa, *sb;
+                if (!next_stage(L::LORA_HALF_TX, lf, sa, sb)) return false;
+                tma_load_2d_pair(sa, &tm_d, lf, c * 64, m_pair * kPairTileM + (int)rank * 128);
+                tma_load_2d_pair(sb, &tm_lb, lf, c * 64, n_blk * kTileN + h * 128 + (int)rank * 64);
+                return true;
+            };
             for (int tile = pair; ok && tile < args.num_tiles; tile += npairs, ++tl) {
                 const int m_pair = tile % args.m_pairs;
                 const int n_blk = tile / args.m_pairs;
@@ -224,32 +262,30 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                     bias_issued |= 1u << bb;
                     bias_par = (bias_par & ~(1u << bb)) | ((((uint32_t)tl >> 1) & 1u) << bb);
                 }
-                const int items = args.k_stages + (lora_on ? lora_chunks_if_on : 0);
-                for (int it = 0; it < items; ++it) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                    const uint32_t lead_full = map_to_rank(smem_u32(&full[stage]), 0);
-                    uint8_t* sa = smem + L::A_OFF + stage * L::A_BYTES;
-                    uint8_t* sb = smem + L::B_OFF + stage * L::B_BYTES;
-                    if (it < args.k_stages) {
-                        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::STAGE_TX);
-                        tma_load_2d_pair(sa, &tm_a, lead_full, it * 128, row_a);
-                        tma_load_2d_pair(sb, &tm_b, lead_full, it * 128, row_b);
-                    } else {
-                        const int c = it - args.k_stages;
-                        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * L::LORA_TX);
-                        tma_load_2d_pair(sa, &tm_d, lead_full, c * 64, row_a);
-                        if constexpr (MODE == Mode::Raw) {
-                            // per N-half, this CTA's 64 of its 128 lora_b rows (64-row boxes)
-                            const int r0 = n_blk * kTileN + (int)rank * 64;
-                            tma_load_2d_pair(sb, &tm_lb, lead_full, c * 64, r0);
-                            tma_load_2d_pair(sb + 64 * 128, &tm_lb, lead_full, c * 64, r0 + 128);
-                        } else {
-                            tma_load_2d_pair(sb, &tm_lb, lead_full, c * 64, row_b);
-                        }
+                // ring items: base stages; raw: the previous tile's LoRA half 1 before base stage
+                // kRawHalf1At (or after the base stages), this tile's half 0 after them; prepared:
+                // the LoRA chunks after the base stages
+                const int h1_at = min(kRawHalf1At, args.k_stages);
+                for (int it = 0; ok && it <= args.k_stages; ++it) {
+                    if (MODE == Mode::Raw && pend && it == h1_at) {
+                        for (int c = 0; ok && c < lora_chunks_if_on; ++c) ok = emit_half(c, 1, prev_m, prev_n);
+                        pend = false;
                     }
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (ok && it < args.k_stages) ok = emit_base(it, row_a, row_b);
+                }
+                if (ok && lora_on) {
+                    if (MODE == Mode::Raw) {
+                        for (int c = 0; ok && c < lora_chunks_if_on; ++c) ok = emit_half(c, 0, m_pair, n_blk);
+                        pend = true;
+                        prev_m = m_pair;
+                        prev_n = n_blk;
+                    } else {
+                        for (int c = 0; ok && c < lora_chunks_if_on; ++c) ok = emit_lora(c, row_a, row_b);
+                    }
                 }
             }
+            if (ok && MODE == Mode::Raw && pend)
+                for (int c = 0; ok && c < lora_chunks_if_on; ++c) ok = emit_half(c, 1, prev_m, prev_n);
             if (!ok || *abort_flag) {
                 // Let this CTA's own-barrier copies land before it can exit (the pair's code-tile
                 // loads complete on the leader's barriers; both CTAs meet at the final cluster
@@ -303,43 +339,44 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             int stage = 0, slot = 0;
             uint32_t phase = 0, slot_use = 0, lacc_waits = 0;
             bool ok = true;
-            // Raw path: LoRA half `half` of a tile from its chunk stages s0 / s1 into the LoRA
-            // accumulator (M = 256, N = 128; each CTA holds 64 of the half's lora_b rows).
-            auto lora_half = [&](int half, int s0, int s1) {
+            // Raw path: one LoRA half of a tile, one ring item per 64-rank chunk (d rows and this
+            // CTA's 64 lora_b rows of the half), into the LoRA accumulator (M = 256, N = 128).
+            auto lora_half = [&]() -> bool {
                 for (int c = 0; c < lora_chunks_if_on; ++c) {
-                    const int stc = (c == 0) ? s0 : s1;
-                    const uint32_t a_addr = smem_u32(smem + L::A_OFF + stc * L::A_BYTES);
-                    const uint32_t b_addr = smem_u32(smem + L::B_OFF + stc * L::B_BYTES) + half * (64 * 128);
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) return false;
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + L::A_OFF + stage * L::A_BYTES);
+                    const uint32_t b_addr = smem_u32(smem + L::B_OFF + stage * L::B_BYTES);
                     const int rem = args.r - c * 64;
                     const int ksteps = rem >= 64 ? 4 : (rem + 15) / 16;
                     for (int j = 0; j < ksteps; ++j)
                         tc_mma_bf16_pair(tmem + T::LACC, sdesc_sw128(a_addr + j * 32), sdesc_sw128(b_addr + j * 32),
                                          IDESC_BF16_HALF, (c > 0 || j > 0) ? 1u : 0u);
+                    tc_commit_pair_multicast(&empty[stage], kBoth);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
+                return true;
             };
-            // Raw path: the previous tile's LoRA half 1 waits until its half 0 has been read; it is
-            // issued a few stages into the next tile (or after its base stages, or at the end), so
-            // the tensor pipe does not idle meanwhile.  Its chunk stages stay held until then.
+            // Raw path: the previous tile's half 1, once the epilogue warps of half 0 (both CTAs)
+            // have read the LoRA accumulator; issued kRawHalf1At stages into the next tile so that
+            // the tensor pipe does not idle meanwhile.
             bool pend = false;
-            int pst0 = 0, pst1 = 0;
             auto finish_pending = [&]() -> bool {
                 if (!mbar_wait_cluster(lacc_empty, (lacc_waits++ & 1) ^ 1, abort_flag)) return false;
                 tc_fence_after();
-                lora_half(1, pst0, pst1);
+                if (!lora_half()) return false;
                 tc_commit_pair_multicast(lacc_full, kBoth);
-                tc_commit_pair_multicast(&empty[pst0], kBoth);
-                if (lora_chunks_if_on > 1) tc_commit_pair_multicast(&empty[pst1], kBoth);
                 pend = false;
                 return true;
             };
-            constexpr int kDeferStages = 2;   // at most 2 of the 4 ring stages hold LoRA chunks
+            const int h1_at = min(kRawHalf1At, args.k_stages);
             int i = 0;
             for (int tile = pair; ok && tile < args.num_tiles; tile += npairs, ++i) {
                 // both CTAs' epilogues have read the previous tile's accumulator
                 if (!mbar_wait_cluster(acc_empty, (i & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int it = 0; ok && it < args.k_stages; ++it) {
-                    if (MODE == Mode::Raw && pend && it == kDeferStages && !finish_pending()) { ok = false; break; }
+                    if (MODE == Mode::Raw && pend && it == h1_at && !finish_pending()) { ok = false; break; }
                     // both CTAs staged this slot's scales, and both CTAs' code tiles landed
                     if (!mbar_wait_cluster(&sf_ready[slot], slot_use & 1u, abort_flag)) { ok = false; break; }
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
@@ -358,6 +395,7 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
+                if (MODE == Mode::Raw && pend && !finish_pending()) { ok = false; break; }   // k_stages <= h1_at
                 if (lora_on && MODE == Mode::Prepared) {
                     // the folded LoRA term into the same accumulator, after the base product
                     for (int c = 0; ok && c < lora_chunks_if_on; ++c) {
@@ -376,23 +414,13 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                     if (!ok) break;
                     tc_commit_pair_multicast(tmem_full, kBoth);   // both CTAs' accumulators are complete
                 } else if (lora_on && MODE == Mode::Raw) {
-                    // raw LoRA term in its own 128-column accumulator, one N-half at a time
-                    if (pend && !finish_pending()) { ok = false; break; }
-                    int st0 = 0, st1 = 0;      // stages of LoRA chunks 0 and 1 (r <= 128)
-                    for (int c = 0; ok && c < lora_chunks_if_on; ++c) {
-                        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-                        if (c == 0) st0 = stage; else st1 = stage;
-                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                    }
-                    // the previous tile's half 1 has been read
-                    if (ok && !mbar_wait_cluster(lacc_empty, (lacc_waits++ & 1) ^ 1, abort_flag)) ok = false;
-                    if (!ok) break;
+                    // raw LoRA half 0 in its own accumulator, once the previous tile's half 1 has
+                    // been read
+                    if (!mbar_wait_cluster(lacc_empty, (lacc_waits++ & 1) ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    lora_half(0, st0, st1);
+                    if (!lora_half()) { ok = false; break; }
                     tc_commit_pair_multicast(tmem_full, kBoth);   // base accumulator + LoRA half 0
                     pend = true;
-                    pst0 = st0;
-                    pst1 = st1;
                 } else {
                     tc_commit_pair_multicast(tmem_full, kBoth);   // both CTAs' accumulators are complete
                 }
@@ -493,12 +521,12 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                 if (h == 1 && !__all_sync(kAll, mbar_wait(lacc_full, i & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t lv[16];
-                    tmem_load_16(tmem + lane_off + T::LACC + c * 16, lv);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t lv[32];
+                    tmem_load_32(tmem + lane_off + T::LACC + c * 32, lv);
                     tmem_load_wait();
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) v[c * 16 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 16 + k]);
+                    for (int k = 0; k < 32; ++k) v[c * 32 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 32 + k]);
                 }
                 tc_fence_before();
                 if (rank == 0) mbar_arrive(lacc_empty);
