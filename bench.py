@@ -426,37 +426,86 @@ def run_cfg4(args, rank, world, device):
 
 
 def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
-    a_h = p.a.pin_memory()
-    a_sf_h = p.a_sf.pin_memory()
-    d_h = p.d.pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    a_d, a_sf_d, d_d = torch.empty_like(st["a"]), torch.empty_like(st["a_sf"]), torch.empty_like(st["d"])
-    h2d = a_h.numel() + a_sf_h.numel() + d_h.numel() * 2
+    """End to end through the public API with host buffers.  Every step copies its activation-side
+    inputs (a, a_sf, d) host -> device from pinned memory, makes the call, and copies out back to
+    pinned host memory.  a's, a_sf's and d's bytes sit in one pinned staging buffer (one copy per
+    step).  When a step moves more than 4 MB, steps are pipelined the way a serving loop would run
+    them: two step slots alternate, and the host -> device copies, the calls and the device -> host
+    copies run on three streams ordered by events, so one step's copies overlap its neighbours'
+    calls.  Smaller steps run on one stream: there the cross-stream hand-offs cost more than the
+    copies."""
+    def region(nbytes):
+        return (nbytes + 255) // 256 * 256
+    na, nsf, nd = p.a.numel(), p.a_sf.numel(), p.d.numel() * 2
+    oa, osf, od = 0, region(na), region(na) + region(nsf)
+    total = od + region(nd)
+    slots = 2
+    host_in, dev_in, views = [], [], []
+    for _ in range(slots):
+        h = torch.empty(total, dtype=torch.uint8).pin_memory()
+        h[oa:oa + na].copy_(p.a.reshape(-1))
+        h[osf:osf + nsf].copy_(p.a_sf.reshape(-1))
+        h[od:od + nd].copy_(p.d.reshape(-1).view(torch.uint8))
+        dbuf = torch.empty(total, dtype=torch.uint8, device=device)
+        host_in.append(h)
+        dev_in.append(dbuf)
+        views.append((dbuf[oa:oa + na].view(p.a.shape), dbuf[osf:osf + nsf].view(p.a_sf.shape),
+                      dbuf[od:od + nd].view(torch.bfloat16).view(p.d.shape)))
+    outs = [torch.empty_like(out) for _ in range(slots)]
+    outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(slots)]
+    h2d = na + nsf + nd
     d2h = out.numel() * 2
+    pipelined = h2d + d2h > (4 << 20)
+    if pipelined:
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    else:
+        s_in = s_out = stream
+    n_ev = steps + 8
+    ev_in = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_call = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_out = [torch.cuda.Event() for _ in range(n_ev)]
 
-    def one():
-        a_d.copy_(a_h, non_blocking=True)
-        a_sf_d.copy_(a_sf_h, non_blocking=True)
-        d_d.copy_(d_h, non_blocking=True)
-        if prepared:
-            L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, lora_adapter=adp, bias=st["bias"], out=out)
-        else:
-            L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, st["lora_b"], s, bias=st["bias"], out=out)
-        out_h.copy_(out, non_blocking=True)
+    def one(i):
+        k = i % slots if pipelined else 0
+        with torch.cuda.stream(s_in):
+            if pipelined and i >= slots:
+                s_in.wait_event(ev_call[i - slots])     # the slot's previous call has read its inputs
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+            if pipelined:
+                ev_in[i].record(s_in)
+        with torch.cuda.stream(stream):
+            if pipelined:
+                stream.wait_event(ev_in[i])
+                if i >= slots:
+                    stream.wait_event(ev_out[i - slots])    # the slot's previous output has been copied out
+            a_d, a_sf_d, d_d = views[k]
+            if prepared:
+                L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, lora_adapter=adp, bias=st["bias"],
+                                out=outs[k])
+            else:
+                L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, st["lora_b"], s, bias=st["bias"],
+                                out=outs[k])
+            if pipelined:
+                ev_call[i].record(stream)
+        with torch.cuda.stream(s_out):
+            if pipelined:
+                s_out.wait_event(ev_call[i])
+            outs_h[k].copy_(outs[k], non_blocking=True)
+            if pipelined:
+                ev_out[i].record(s_out)
 
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            one()
-        torch.cuda.synchronize(device)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            one()
-        e1.record(stream)
+    for i in range(4):
+        one(i)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(steps):
+        one(i + 4)
+    e1.record(s_out)
     torch.cuda.synchronize(device)
     ms = e0.elapsed_time(e1) / steps
-    return dict(ms_step=ms, steps=steps, h2d=h2d, d2h=d2h)
+    return dict(ms_step=ms, steps=steps, h2d=h2d, d2h=d2h, pipelined=pipelined)
 
 
 # ---------------------------------------------------------------------------------------
@@ -633,7 +682,7 @@ def main():
         "config": config_block(args, c), "roofline": roof, "clocks": res["clocks"],
         "e2e": {"value": whole_job(e2e_val, world), "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"],
-                "note": "per step: a, a_sf, d host->device (pinned), call, out device->host; weights resident"},
+                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; " + ("two step slots pipelined over three streams" if res["e2e"].get("pipelined") else "one stream") + "; weights resident"},
         "gpu_launches": res["launches"],
         "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
         "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],
