@@ -429,11 +429,10 @@ def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
     """End to end through the public API with host buffers.  Every step copies its activation-side
     inputs (a, a_sf, d) host -> device from pinned memory, makes the call, and copies out back to
     pinned host memory.  a's, a_sf's and d's bytes sit in one pinned staging buffer (one copy per
-    step).  When a step moves more than 4 MB, steps are pipelined the way a serving loop would run
-    them: two step slots alternate, and the host -> device copies, the calls and the device -> host
-    copies run on three streams ordered by events, so one step's copies overlap its neighbours'
-    calls.  Smaller steps run on one stream: there the cross-stream hand-offs cost more than the
-    copies."""
+    step).  Steps are pipelined the way a serving loop would run them: two step slots alternate,
+    and the host -> device copies, the calls and the device -> host copies run on three streams
+    ordered by events, so one step's copies overlap its neighbours' calls.  The timed steps are
+    replayed from one CUDA graph."""
     def region(nbytes):
         return (nbytes + 255) // 256 * 256
     na, nsf, nd = p.a.numel(), p.a_sf.numel(), p.d.numel() * 2
@@ -455,7 +454,7 @@ def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
     outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(slots)]
     h2d = na + nsf + nd
     d2h = out.numel() * 2
-    pipelined = h2d + d2h > (4 << 20)
+    pipelined = True
     if pipelined:
         s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     else:
@@ -465,10 +464,11 @@ def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
     ev_call = [torch.cuda.Event() for _ in range(n_ev)]
     ev_out = [torch.cuda.Event() for _ in range(n_ev)]
 
-    def one(i):
+    def one(i, first):
+        # waits only on events of this batch of steps (a captured batch cannot wait on the others)
         k = i % slots if pipelined else 0
         with torch.cuda.stream(s_in):
-            if pipelined and i >= slots:
+            if pipelined and i - first >= slots:
                 s_in.wait_event(ev_call[i - slots])     # the slot's previous call has read its inputs
             dev_in[k].copy_(host_in[k], non_blocking=True)
             if pipelined:
@@ -476,7 +476,7 @@ def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
         with torch.cuda.stream(stream):
             if pipelined:
                 stream.wait_event(ev_in[i])
-                if i >= slots:
+                if i - first >= slots:
                     stream.wait_event(ev_out[i - slots])    # the slot's previous output has been copied out
             a_d, a_sf_d, d_d = views[k]
             if prepared:
@@ -495,16 +495,35 @@ def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
                 ev_out[i].record(s_out)
 
     for i in range(4):
-        one(i)
+        one(i, 0)
+    torch.cuda.synchronize(device)
+    # the steps are captured in one CUDA graph (copies, calls, and on the pipelined path the
+    # cross-stream orderings), so the host issues one launch instead of a Python loop per step
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        if pipelined:
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            s_in.wait_event(fork)
+            s_out.wait_event(fork)
+        for i in range(steps):
+            one(i + 4, 4)
+        if pipelined:
+            for st_ in (s_in, s_out):
+                join = torch.cuda.Event()
+                join.record(st_)
+                stream.wait_event(join)
+    g.replay()
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    for i in range(steps):
-        one(i + 4)
-    e1.record(s_out)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
     torch.cuda.synchronize(device)
     ms = e0.elapsed_time(e1) / steps
+    del g
     return dict(ms_step=ms, steps=steps, h2d=h2d, d2h=d2h, pipelined=pipelined)
 
 
@@ -682,7 +701,7 @@ def main():
         "config": config_block(args, c), "roofline": roof, "clocks": res["clocks"],
         "e2e": {"value": whole_job(e2e_val, world), "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"],
-                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; " + ("two step slots pipelined over three streams" if res["e2e"].get("pipelined") else "one stream") + "; weights resident"},
+                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; two step slots pipelined over three streams; the steps captured in one CUDA graph; weights resident"},
         "gpu_launches": res["launches"],
         "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
         "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],
