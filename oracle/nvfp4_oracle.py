@@ -17,6 +17,8 @@ It restates, slowly and in float64, what the pages define:
 * ``flashinfer.gemm.prepare_nvfp4_lora_adapter`` -- summary paragraph (the fold:
   ``ratio = div.rn.f32(lora_scale, alpha[0])``,
   ``b_folded[i] = bf16_rne(fp32(lora_b[i]) * ratio)``).
+* the quantizer the mm_nvfp4_lora page names as the producer of a / a_sf (``fp4_quantize``),
+  by the reading given at :func:`quantize_nvfp4`.
 
 Readings taken where the pages are silent (each is listed in the design doc):
 
@@ -313,6 +315,84 @@ def eager_prepare_check(lora_scale: float, alpha: float) -> None:
         raise ValueError("alpha == 0: lora_scale / alpha is undefined")
     if not np.isfinite(fold_ratio(lora_scale, alpha)):
         raise ValueError("lora_scale / alpha is not finite")
+
+
+# --------------------------------------------------------------------------------------
+# The quantizer that produces a and a_sf (mm_nvfp4_lora page: the paragraph after the formula
+# says the operands come "in the 128x4 swizzled layout produced by fp4_quantize()"; Parameters:
+# alpha is "alpha_base / (a_global_scale * b_global_scale)", so dequant(codes, scales) carries
+# a per-tensor global scale).  The pages name the quantizer but not its rule.  The reading
+# taken (listed in the design doc), each step in float32 as the kernel computes it:
+#   per 16-element block along K:  amax = max |x|                (x: bf16, exact in float32)
+#   sf    = E4M3(rne, saturate to 448)( (amax * gs) / 6 )         (6 = largest E2M1 value)
+#   inv   = gs / value(sf)               (sf == 0: every code of the block is +0)
+#   code  = E2M1(rne, saturate to 6)( x * inv ),  sign kept, -0 for negatives rounding to 0
+# so that value(code) * value(sf) / gs ~= x; scale rows past the last row are 0.
+# --------------------------------------------------------------------------------------
+
+#: the 127 finite non-negative E4M3 values, by code 0x00..0x7E
+_E4M3_VALUES = decode_ue4m3(np.arange(0x7F, dtype=np.uint8))
+
+
+def _round_to_table(v: np.ndarray, values: np.ndarray) -> np.ndarray:
+    """Index of the nearest entry of the increasing table `values` to each v >= 0; a tie goes
+    to the even index (the code whose last bit is 0); v above the last entry saturates."""
+    v = np.asarray(v, dtype=np.float64)
+    hi = np.searchsorted(values, v, side="left")          # first entry >= v
+    hi = np.minimum(hi, len(values) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = v - values[lo]
+    d_hi = values[hi] - v
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    idx = np.where(pick_hi, hi, lo)
+    idx = np.where(v >= values[-1], len(values) - 1, idx)
+    return idx
+
+
+def e4m3_rne_satfinite(v: np.ndarray) -> np.ndarray:
+    """float32 v >= 0 -> E4M3 code (round to nearest, ties to even, saturating at 448)."""
+    v = np.asarray(v, dtype=np.float32)
+    if np.any(~np.isfinite(v)) or np.any(v < 0):
+        raise ValueError("scale input must be finite and non-negative")
+    return _round_to_table(v.astype(np.float64), _E4M3_VALUES).astype(np.uint8)
+
+
+def e2m1_rne_satfinite(q: np.ndarray) -> np.ndarray:
+    """float32 q -> 4-bit E2M1 code: magnitude rounded to nearest (ties to even code), saturating
+    at 6; bit 3 holds the sign (so a negative q that rounds to 0 gives -0, code 8)."""
+    q = np.asarray(q, dtype=np.float32)
+    if np.any(~np.isfinite(q)):
+        raise ValueError("non-finite value to quantize")
+    mag = _round_to_table(np.abs(q).astype(np.float64), E2M1_TABLE[:8]).astype(np.uint8)
+    sign = np.signbit(q).astype(np.uint8) << 3
+    return mag | sign
+
+
+def quantize_nvfp4(x_bits: np.ndarray, global_scale: float):
+    """bf16 bit patterns ``[R, K]`` -> (codes ``uint8 [R, K/2]``, swizzled scales of
+    ``sf_buffer_bytes(R, K)`` bytes), by the reading above.  K must be a multiple of 64."""
+    x_bits = np.asarray(x_bits, dtype=np.uint16)
+    rows, k = x_bits.shape
+    if k % 64 != 0:
+        raise ValueError("K must be a multiple of 64")
+    gs = np.float32(global_scale)
+    if not np.isfinite(gs) or gs <= 0:
+        raise ValueError("global_scale must be positive and finite")
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32)            # exact bf16 -> fp32
+    if np.any(~np.isfinite(x)):
+        raise ValueError("non-finite input")
+    blocks = x.reshape(rows, k // SF_VEC, SF_VEC)
+    amax = np.max(np.abs(blocks), axis=2)                                # float32, exact
+    sval = np.float32(amax * gs) / np.float32(6.0)                       # two float32 roundings
+    sf = e4m3_rne_satfinite(sval)                                        # [rows, k/16] codes
+    sfv = _E4M3_VALUES[sf].astype(np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(sfv > 0, gs / np.where(sfv > 0, sfv, np.float32(1)), np.float32(0))
+    q = (blocks * inv.astype(np.float32)[..., None]).astype(np.float32)  # float32 product
+    codes = e2m1_rne_satfinite(q)
+    codes = np.where((sfv > 0)[..., None], codes, np.uint8(0)).reshape(rows, k)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return packed, swizzle_scales(sf, k, pad_value=0)
 
 
 # --------------------------------------------------------------------------------------

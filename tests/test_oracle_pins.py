@@ -379,3 +379,125 @@ def test_measures():
     assert O.sqnr_db(y, y) == float("inf")
     assert abs(O.sqnr_db(y, y + np.array([0.0, 0.0, 0.21])) - 10 * np.log10(21 / 0.0441)) < 1e-9
     np.testing.assert_array_equal(O.tolerance(y), 2.0 ** -7 * np.abs(y) + 2.0 ** -10 * 4.0)
+
+
+# ---------------------------------------------------------------------------------------
+# the quantizer (the reading of fp4_quantize: per-16-block amax, UE4M3 scale, E2M1 codes)
+# ---------------------------------------------------------------------------------------
+
+def _e2m1_nearest_even_brute(q: float) -> int:
+    """Brute force over the 8 magnitudes: nearest, ties to the even code, saturate at 6."""
+    mag = abs(q)
+    best, best_d = 0, None
+    for code in range(8):
+        d = abs(e2m1_closed_form(code) - mag)
+        if best_d is None or d < best_d or (d == best_d and code % 2 == 0):
+            best, best_d = code, d
+    if mag >= 6.0:
+        best = 7
+    return best | (8 if math.copysign(1.0, q) < 0 else 0)
+
+
+def test_e2m1_rounding_matches_brute_force():
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0]
+    vals = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, 6.5, 9.0, 1e30, 0.1, 0.2499, 0.2501, 2.9, 4.99, 5.01]
+    qs = []
+    for v in mids + vals:
+        qs += [v, -v, np.nextafter(np.float32(v), np.float32(0)), np.nextafter(np.float32(v), np.float32(1e38))]
+    qs = np.array(qs, dtype=np.float32)
+    got = O.e2m1_rne_satfinite(qs)
+    want = np.array([_e2m1_nearest_even_brute(float(q)) for q in qs], dtype=np.uint8)
+    np.testing.assert_array_equal(got, want)
+    # the ties, written out from the format: 0.25 -> 0, 0.75 -> 1.0, 1.25 -> 1.0, 1.75 -> 2,
+    # 2.5 -> 2, 3.5 -> 4, 5 -> 4; a negative value that rounds to 0 keeps its sign (-0 = code 8)
+    np.testing.assert_array_equal(O.e2m1_rne_satfinite(np.array(mids[:7], dtype=np.float32)),
+                                  np.array([0, 2, 2, 4, 4, 6, 6], dtype=np.uint8))
+    assert O.e2m1_rne_satfinite(np.array([-0.2], dtype=np.float32))[0] == 8
+
+
+def test_e4m3_rounding_matches_torch_float8_in_range():
+    vals = O.decode_ue4m3(np.arange(0x7F, dtype=np.uint8))
+    mids = (vals[1:] + vals[:-1]) / 2
+    rng = np.random.default_rng(4)
+    x = np.concatenate([vals, mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9),
+                        rng.uniform(0, 448, 4000), np.exp2(rng.uniform(-12, 8.8, 4000))])
+    x = x[x <= 448].astype(np.float32)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.e4m3_rne_satfinite(x), want)
+
+
+def test_e4m3_saturation_and_underflow():
+    x = np.array([448.0, 449.0, 464.0, 465.0, 1e20, 0.0, 2.0 ** -10, 3 * 2.0 ** -10, 2.0 ** -9], dtype=np.float32)
+    np.testing.assert_array_equal(O.e4m3_rne_satfinite(x),
+                                  np.array([0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0, 0, 2, 1], dtype=np.uint8))
+
+
+def _bf16_bits(x64: np.ndarray) -> np.ndarray:
+    x32 = np.asarray(x64, dtype=np.float32)
+    bits = x32.view(np.uint32)
+    assert np.all((bits & 0xFFFF) == 0), "value not exactly representable in bf16"
+    return (bits >> 16).astype(np.uint16)
+
+
+def _round_bf16_bits(x64: np.ndarray) -> np.ndarray:
+    """Round to bf16 through PyTorch (a route independent of the oracle)."""
+    t = torch.from_numpy(np.asarray(x64, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("rows,k", [(1, 64), (130, 256), (256, 512)])
+def test_quantize_round_trip_exact(rows, k):
+    """x built as code * scale / gs with one |6| code per block (so the block's amax fixes the
+    scale exactly) quantizes back to the same codes and scale bytes."""
+    rng = np.random.default_rng(rows + k)
+    nb = k // 16
+    codes = rng.integers(0, 16, size=(rows, k)).astype(np.uint8)
+    codes[:, ::16] = np.where(rng.random((rows, nb)) < 0.5, 7, 15)       # a +-6 in every block
+    sf = rng.integers(0x20, 0x60, size=(rows, nb)).astype(np.uint8)      # 2**-3 .. 2**4
+    gs = 2.0 ** 5
+    vals = np.array([e2m1_closed_form(c) for c in range(16)])[codes]
+    x = vals * np.repeat(ue4m3_library(sf.ravel()).reshape(rows, nb), 16, axis=1) / gs
+    packed, sf_buf = O.quantize_nvfp4(_bf16_bits(x), gs)
+    codes_back = np.empty((rows, k), dtype=np.uint8)
+    codes_back[:, 0::2] = packed & 0x0F
+    codes_back[:, 1::2] = packed >> 4
+    np.testing.assert_array_equal(O.unswizzle_scales(sf_buf, rows, k), sf)
+    # codes 0 (+0) and 8 (-0) come back as they went in: the sign of a zero survives
+    np.testing.assert_array_equal(codes_back, codes)
+
+
+def test_quantize_zero_block_saturation_and_padding():
+    rows, k = 3, 64
+    x = np.zeros((rows, k), dtype=np.float64)
+    x[1, :16] = 1.0e4              # amax * gs / 6 far above 448: scale saturates, codes saturate
+    x[1, 5] = -3.0e4
+    x[2, 16:32] = np.linspace(-1, 1, 16)
+    packed, sf_buf = O.quantize_nvfp4(_round_bf16_bits(x), 1.0)
+    sf = O.unswizzle_scales(sf_buf, rows, k)
+    assert sf[0].tolist() == [0, 0, 0, 0] and packed[0].tolist() == [0] * 32
+    assert sf[1, 0] == 0x7E
+    lo, hi = packed[1, :8] & 0x0F, packed[1, :8] >> 4
+    blk = np.empty(16, dtype=np.uint8)
+    blk[0::2], blk[1::2] = lo, hi
+    assert blk[5] == 15 and np.all(np.delete(blk, 5) == 7)        # -6 and +6 (saturated)
+    # scale bytes of the padded rows 3..127 are 0
+    full = np.frombuffer(sf_buf.tobytes(), dtype=np.uint8)
+    mask = np.ones(full.size, dtype=bool)
+    rr, cc = np.meshgrid(np.arange(rows), np.arange(k // 16), indexing="ij")
+    mask[O.sf_offset(rr, cc, k)] = False
+    assert np.all(full[mask] == 0)
+
+
+def test_quantize_error_bound_random():
+    """dequant(quant(x)) / gs stays within amax/6 * (1 + 2**-3) of x in every block."""
+    rng = np.random.default_rng(9)
+    rows, k = 64, 256
+    x = rng.standard_normal((rows, k)) * np.exp2(rng.integers(-6, 6, size=(rows, 1)))
+    xb = _round_bf16_bits(x)
+    xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    amax = np.abs(xf).max()
+    gs = 448.0 * 6.0 / amax
+    packed, sf_buf = O.quantize_nvfp4(xb, gs)
+    back = O.dequant(packed, sf_buf, rows, k) / np.float32(gs)
+    blk_amax = np.repeat(np.abs(xf).reshape(rows, k // 16, 16).max(axis=2), 16, axis=1)
+    assert np.all(np.abs(back - xf) <= blk_amax / 6.0 * (1 + 2.0 ** -3))
