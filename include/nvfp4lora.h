@@ -181,6 +181,28 @@ NVFP4LORA_API nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream);
  */
 NVFP4LORA_API nvfp4lora_status nvfp4lora_selftest_wait_timeout(int64_t limit_ns, nvfp4lora_stream stream);
 
+/*
+ * NVFP4 quantizer: the producer of a / a_sf that the mm_nvfp4_lora page names (the paragraph
+ * after the formula: "... in the 128x4 swizzled layout produced by fp4_quantize()"; Parameters:
+ * alpha = alpha_base / (a_global_scale * b_global_scale)).  The pages give no rule; this library
+ * computes, per 16-element block along K, in float32:
+ *     amax = max |x|;  sf = E4M3(rne, saturating at 448)((amax * gs) / 6);
+ *     code = E2M1(rne, saturating at 6)(x * (gs / value(sf)))   (sf == 0: +0 codes),
+ * so value(code) * value(sf) / gs approximates x.
+ *   x       bf16 [rows, K] device, row-major, 16-byte aligned.  Finite values.
+ *   global_scale  fp32 [1] device: gs, positive and finite (read on the device; no host read).
+ *   codes   uint8 [rows, K/2] device, caller-owned, 16-byte aligned: element 2j of a row in the
+ *           low nibble of byte j.
+ *   scales  uint8 device, caller-owned, 16-byte aligned, scales_bytes >= ceil(rows/128)*128*(K/16):
+ *           the 128x4 swizzled layout; the bytes of padded rows are written as 0.
+ * K % 64 == 0 (whole scale atoms).  Enqueued on `stream`; NVFP4LORA_ERR_INVALID_ARG (nothing
+ * enqueued) for a rule violation.  The pages have no counterpart for the exact rule.
+ */
+NVFP4LORA_API nvfp4lora_status nvfp4lora_quantize(
+    const uint16_t* x, int64_t rows, int64_t K, const float* global_scale,
+    uint8_t* codes, uint8_t* scales, int64_t scales_bytes,
+    nvfp4lora_stream stream);
+
 /* Message of the last failing call on this host thread ("" when none). */
 NVFP4LORA_API const char* nvfp4lora_last_error(void);
 

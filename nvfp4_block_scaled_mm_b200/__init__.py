@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4lor
 __all__ = [
     "StaleAdapterError", "PreparedNvFp4LoraAdapter", "mm_nvfp4_lora", "prepare_nvfp4_lora_adapter",
     "nvfp4lora_mm", "nvfp4lora_prepare", "nvfp4lora_refold", "nvfp4lora_mm_prepared",
-    "nvfp4lora_device_status", "library_path", "version",
+    "nvfp4lora_device_status", "nvfp4lora_quantize", "fp4_quantize", "library_path", "version",
 ]
 
 OK, INVALID_ARG, STALE, ALPHA_ZERO, UNSUPPORTED_ARCH, DEVICE_TIMEOUT, CUDA_ERR = range(7)
@@ -63,6 +63,8 @@ def _load():
     lib.nvfp4lora_device_status.restype = ctypes.c_int
     lib.nvfp4lora_selftest_wait_timeout.argtypes = [I64, P]
     lib.nvfp4lora_selftest_wait_timeout.restype = ctypes.c_int
+    lib.nvfp4lora_quantize.argtypes = [P, I64, I64, P, P, P, I64, P]
+    lib.nvfp4lora_quantize.restype = ctypes.c_int
     lib.nvfp4lora_last_error.argtypes = []
     lib.nvfp4lora_last_error.restype = ctypes.c_char_p
     lib.nvfp4lora_version.argtypes = []
@@ -170,6 +172,12 @@ def nvfp4lora_mm_prepared(a, b, a_sf, b_sf, alpha, d, adp, cur_lora_b, cur_lora_
 def nvfp4lora_device_status(stream=None) -> None:
     """Synchronise the stream and raise DeviceTimeoutError if a kernel's wait ran out."""
     _check(_lib.nvfp4lora_device_status(_stream(stream)))
+
+
+def nvfp4lora_quantize(x, rows, K, global_scale, codes, scales, stream=None):
+    _check(_lib.nvfp4lora_quantize(_ptr(x), int(rows), int(K), _ptr(global_scale), _ptr(codes), _ptr(scales),
+                                   scales.numel(), _stream(stream)))
+    return codes, scales
 
 
 def nvfp4lora_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
@@ -319,3 +327,34 @@ def mm_nvfp4_lora(a: torch.Tensor, b: torch.Tensor, a_sf: torch.Tensor, b_sf: to
             raise ValueError(f"d must be [M, r] and lora_b [N, r]; got {tuple(d.shape)}, {tuple(lora_b.shape)}")
         nvfp4lora_mm(a, b, a_sf, b_sf, alpha, d, lora_b, lora_scale, r, bias, out, M, N, K, stream)
         return out
+
+
+def fp4_quantize(x: torch.Tensor, global_scale: torch.Tensor, *, codes: Optional[torch.Tensor] = None,
+                 scales: Optional[torch.Tensor] = None):
+    """Quantize bf16 ``x [rows, K]`` into the operand format of :func:`mm_nvfp4_lora`: E2M1
+    ``codes uint8 [rows, K/2]`` and UE4M3 ``scales`` (16 K-elements each, 128x4 swizzled, rows
+    padded to 128), with the per-tensor ``global_scale`` (fp32, one element, on the device) folded
+    in: ``value(code) * value(scale) / global_scale`` approximates x.  Rule (per 16-block, fp32):
+    ``scale = e4m3(amax * gs / 6)``, ``code = e2m1(x * gs / value(scale))``, round to nearest
+    even, saturating."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(global_scale, "global_scale", torch.float32)
+    if global_scale.numel() != 1:
+        raise ValueError("global_scale must be a one-element fp32 tensor")
+    rows, K = x.shape
+    if K % 64 != 0:
+        raise ValueError(f"K = {K}: a multiple of 64 is required")
+    nbytes = (rows + 127) // 128 * 128 * (K // 16)
+    if codes is None:
+        codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=x.device)
+    else:
+        _need(codes, "codes", torch.uint8, 2)
+        if tuple(codes.shape) != (rows, K // 2):
+            raise ValueError(f"codes must be [rows, K/2] = [{rows}, {K // 2}]")
+    if scales is None:
+        scales = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    else:
+        _need(scales, "scales", torch.uint8)
+    with torch.cuda.device(x.device):
+        nvfp4lora_quantize(x, rows, K, global_scale, codes, scales, torch.cuda.current_stream(x.device))
+    return codes, scales

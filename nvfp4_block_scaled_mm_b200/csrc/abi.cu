@@ -27,6 +27,7 @@
 #include "gemm_decode.cuh"
 #include "gemm_pair.cuh"
 #include "ptx.cuh"
+#include "quantize.cuh"
 #include "selftest.cuh"
 
 namespace nvfp4lora {
@@ -691,6 +692,36 @@ nvfp4lora_status nvfp4lora_selftest_wait_timeout(int64_t limit_ns, nvfp4lora_str
         (unsigned long long)limit_ns);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return NVFP4LORA_OK;
+}
+
+nvfp4lora_status nvfp4lora_quantize(const uint16_t* x, int64_t rows, int64_t K, const float* global_scale,
+                                    uint8_t* codes, uint8_t* scales, int64_t scales_bytes, nvfp4lora_stream stream) {
+    t_last_error.clear();
+    if (!x || !global_scale || !codes || !scales)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "x, global_scale, codes and scales must be non-null");
+    if (rows < 1 || K < 64 || K % 64 != 0)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "rows >= 1 and K >= 64 with K %% 64 == 0 are required (rows=%lld K=%lld)",
+                    (long long)rows, (long long)K);
+    if (rows > (int64_t)1 << 40 || K > (int64_t)1 << 30)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "rows x K too large");
+    const int64_t need = (rows + 127) / 128 * 128 * (K / 16);
+    if (scales_bytes < need)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "scales needs %lld bytes (rows padded to 128 x K/16), got %lld",
+                    (long long)need, (long long)scales_bytes);
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "x, codes and scales must be 16-byte aligned");
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+    const int64_t total = (rows + 127) / 128 * 128 * (K / 16);             // one thread per block
+    const int64_t want = (total + kQuantThreads - 1) / kQuantThreads;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)info->sms * 8));
+    quantize_kernel<<<grid, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, rows, K, global_scale,
+                                                                                          codes, scales);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
     return NVFP4LORA_OK;
 }
 

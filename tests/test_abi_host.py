@@ -116,3 +116,22 @@ def test_selftest_limit_is_checked_before_cuda(lib):
     for bad in (0, -5, 2_000_000_000):
         assert f(bad, None) == 1
         assert b"limit_ns" in lib.nvfp4lora_last_error()
+
+
+def test_quantize_rules_are_checked_before_cuda(lib):
+    f = lib.nvfp4lora_quantize
+    f.restype = ctypes.c_int
+    f.argtypes = [P, I64, I64, P, P, P, I64, P]
+    lib.nvfp4lora_last_error.restype = ctypes.c_char_p
+    ok = dict(x=0x10000, rows=130, K=256, gs=0x20000, codes=0x30000, scales=0x40000, nbytes=256 * 16)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["x"], a["rows"], a["K"], a["gs"], a["codes"], a["scales"], a["nbytes"], None)
+
+    for bad, word in ((dict(K=96), b"K"), (dict(K=0), b"K"), (dict(rows=0), b"rows"),
+                      (dict(nbytes=256 * 16 - 1), b"scales needs"), (dict(x=0x10008), b"aligned"),
+                      (dict(scales=None), b"non-null"), (dict(gs=None), b"non-null")):
+        assert call(**bad) == 1, bad
+        assert word in lib.nvfp4lora_last_error(), (bad, lib.nvfp4lora_last_error())
