@@ -41,11 +41,16 @@ WORKLOADS = {
     "cfg2": dict(src="cfg2", steps=2000),
     "cfg3": dict(src="cfg3", steps=100),
     "cfg4": dict(src=None, steps=None),   # adapter-switch sweep (its own runner)
+    "quant": dict(src=None, steps=400),   # the NVFP4 quantizer on the cfg3 activations (its own runner)
 }
+
+QUANT_ROWS, QUANT_K = 8192, 8192         # cfg3's a: M x K
 
 
 def describe(name):
     from workloads import CFG4, CONFIGS
+    if name == "quant":
+        return dict(rows=QUANT_ROWS, K=QUANT_K, seed=5)
     if name == "cfg4":
         # the sweep's headline point (the reference arm times the oracle on it)
         return dict(M=CFG4["Ms"][0], N=CFG4["N"], K=CFG4["K"], r=CFG4["rs"][0], path="raw",
@@ -425,6 +430,89 @@ def run_cfg4(args, rank, world, device):
     return 0
 
 
+def run_quant(args, rank, world, device):
+    """The NVFP4 quantizer (fp4_quantize reading) on bf16 activations of cfg3's shape: HBM-bound,
+    2 bytes read and 0.5 + 1/16 written per element.  Inputs rotate through copies totalling
+    >= 3x L2; K calls in one CUDA graph, timed with CUDA events."""
+    import nvfp4_block_scaled_mm_b200 as L
+    rows, K = QUANT_ROWS, QUANT_K
+    g = torch.Generator().manual_seed(5 + 1000 * rank)
+    x = (torch.randn(rows, K, generator=g) * 2.0).to(torch.bfloat16)
+    gs_v = 448.0 * 6.0 / x.float().abs().max().item()
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(1, math.ceil(3 * l2 / (x.numel() * 2)))
+    xs = [x.to(device) for _ in range(copies)]
+    gs = torch.tensor([gs_v], dtype=torch.float32, device=device)
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((rows + 127) // 128 * 128 * (K // 16), dtype=torch.uint8, device=device)
+    nbytes = rows * K * 2 + rows * K // 2 + scales.numel() + 4
+    steps = args.steps if args.steps is not None else WORKLOADS["quant"]["steps"]
+    stream = torch.cuda.Stream(device)
+
+    def step(i):
+        L.fp4_quantize(xs[i % copies], gs, codes=codes, scales=scales)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+        g_run = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_run, stream=stream):
+            for i in range(steps):
+                step(i)
+    g_run.replay()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g_run.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+    L.nvfp4lora_device_status(stream)
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        ms = max_over_ranks(ms, device)
+    value = nbytes / (ms * 1e-3) / 1e9
+    peaks, peak_src = measured_peaks()
+    line = {
+        "metric": METRIC, "value": whole_job(value, world), "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 -> nvfp4 (e2m1 codes + ue4m3 scales)", "data": "synthetic",
+        "config": {"workload": f"quant: NVFP4 quantizer, bf16 [{rows}, {K}] (cfg3's activations) -> codes + scales",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2_defeat": "inputs rotate through copies totalling >= 3x L2",
+                   "timing": "CUDA graph of K back-to-back calls, CUDA events on the launching stream"},
+        "roofline": {"bound": "hbm", "achieved": value, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": value / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}", "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes},
+        "clocks": clk.summary(),
+        "e2e": {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+                "note": "not measured for the quantizer; the end-to-end figures are the GEMM lines'"},
+        "gpu_launches": steps,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import time
+        import oracle as O
+        xb = x[:64].view(torch.int16).numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < 10.0:
+            O.quantize_nvfp4(xb, gs_v)
+            n += 1
+        dt = (time.perf_counter() - t0) / n
+        frac = 64 / rows
+        line["cpu_baseline"] = {"value": nbytes * frac / dt / 1e9, "unit": "GB/s", "cores": torch.get_num_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} x oracle quantizer on the first 64 of {rows} rows "
+                                          f"({frac:.4f} of the workload each), {n * dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
     """End to end through the public API with host buffers.  Every step copies its activation-side
     inputs (a, a_sf, d) host -> device from pinned memory, makes the call, and copies out back to
@@ -605,6 +693,8 @@ def run_reference(args, rank, world):
     from workloads import make_problem
     if rank != 0:
         return 0
+    if args.workload == "quant":
+        return run_reference_quant(args)
     c = describe(args.workload)
     p = make_problem(c["M"], c["N"], c["K"], c["r"], c["seed"], alpha=c["alpha"],
                      lora_scale=c["lora_scale"], bias=c["bias"])
@@ -631,6 +721,38 @@ def run_reference(args, rank, world):
                          "sample": f"each step: oracle on all {c['M']} rows x the first {ncols} of {c['N']} "
                                    f"output columns ({ncols / c['N']:.4f} of the workload)"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_quant(args):
+    """Reference arm of the quantizer workload: the oracle quantizer on a bounded row sample."""
+    import oracle as O
+    c = describe("quant")
+    rows, K = c["rows"], c["K"]
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(rows, K, generator=g) * 2.0).to(torch.bfloat16)
+    gs_v = 448.0 * 6.0 / x.float().abs().max().item()
+    nrows = 64
+    xb = x[:nrows].view(torch.int16).numpy().view(np.uint16)
+    nbytes = rows * K * 2 + rows * K // 2 + (rows + 127) // 128 * 128 * (K // 16) + 4
+    K_steps = args.steps if args.steps is not None else 20
+    for _ in range(args.warmup):
+        O.quantize_nvfp4(xb, gs_v)
+    t0 = time.perf_counter()
+    for _ in range(K_steps):
+        O.quantize_nvfp4(xb, gs_v)
+    ms_step = (time.perf_counter() - t0) / K_steps * 1e3
+    value = nbytes * nrows / rows / (ms_step * 1e-3) / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"quant: NVFP4 quantizer, bf16 [{rows}, {K}] (cfg3's activations) -> codes + scales"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": f"each step: oracle quantizer on the first {nrows} of {rows} rows"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -671,8 +793,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", device_id=device,
                                              timeout=datetime.timedelta(seconds=120))
-    if args.workload == "cfg4":
-        rc = run_cfg4(args, rank, world, device)
+    if args.workload in ("cfg4", "quant"):
+        rc = (run_cfg4 if args.workload == "cfg4" else run_quant)(args, rank, world, device)
         if world > 1:
             torch.distributed.destroy_process_group()
         return rc

@@ -715,8 +715,9 @@ nvfp4lora_status nvfp4lora_quantize(const uint16_t* x, int64_t rows, int64_t K, 
     DeviceInfo* info = nullptr;
     nvfp4lora_status st = device_info(&dev, &info);
     if (st != NVFP4LORA_OK) return st;
-    const int64_t total = (rows + 127) / 128 * 128 * (K / 16);             // one thread per block
+    const int64_t total = (rows + 127) / 128 * 128 * (K / 16);             // one thread per block per step
     const int64_t want = (total + kQuantThreads - 1) / kQuantThreads;
+    // a grid-stride loop over one wave: the launch bounds keep 8 CTAs resident per SM
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)info->sms * 8));
     quantize_kernel<<<grid, kQuantThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, rows, K, global_scale,
                                                                                           codes, scales);

@@ -47,13 +47,41 @@ __device__ __forceinline__ uint32_t e2m1x2_rn_satfinite(float lo, float hi) {
     return out;
 }
 
-__global__ void __launch_bounds__(kQuantThreads)
+// One 16-element block: amax, scale byte, 16 codes (8 bytes); `w` holds the block's 16 bf16.
+__device__ __forceinline__ uint32_t quantize_block(const uint4 w0, const uint4 w1, float gs, uint2& packed_out) {
+    const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float v[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(wv[i] << 16);
+        v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        amax = fmaxf(amax, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
+    }
+    const uint32_t sfb = e4m3_rn_satfinite(__fdiv_rn(__fmul_rn(amax, gs), 6.0f));
+    uint32_t packed[2] = {0u, 0u};
+    const float sfv = e4m3_value(sfb);
+    if (sfv > 0.0f) {
+        const float inv = __fdiv_rn(gs, sfv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t byte = e2m1x2_rn_satfinite(__fmul_rn(v[2 * i], inv), __fmul_rn(v[2 * i + 1], inv));
+            packed[i >> 2] |= byte << ((i & 3) * 8);
+        }
+    }
+    packed_out = make_uint2(packed[0], packed[1]);
+    return sfb;
+}
+
+// One thread per 16-element block per step; launch bounds for 8 resident CTAs (64 warps) per SM,
+// so that enough loads are in flight to cover the memory latency.
+__global__ void __launch_bounds__(kQuantThreads, 8)
 quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, const float* __restrict__ gs_ptr,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
     const float gs = *gs_ptr;
     const int64_t nb = k / 16;                               // blocks per row (a multiple of 4)
     const int64_t rows_p = (rows + 127) / 128 * 128;
-    const int64_t total = rows_p * nb;                       // a multiple of 4 and of 128 * 4
+    const int64_t total = rows_p * nb;                       // a multiple of 4
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;  // a multiple of 32
     const int lane = threadIdx.x & 31;
     // every lane runs the same number of iterations, so the shuffles below see a full warp
@@ -65,28 +93,9 @@ quantize_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, const f
         uint32_t sfb = 0;
         if (live && r < rows) {
             const uint4* src = reinterpret_cast<const uint4*>(x + r * k + c * 16);
-            const uint4 w0 = __ldg(src), w1 = __ldg(src + 1);
-            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            float v[16];
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                v[2 * i] = __uint_as_float(wv[i] << 16);
-                v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-                amax = fmaxf(amax, fmaxf(fabsf(v[2 * i]), fabsf(v[2 * i + 1])));
-            }
-            sfb = e4m3_rn_satfinite(__fdiv_rn(__fmul_rn(amax, gs), 6.0f));
-            uint32_t packed[2] = {0u, 0u};
-            const float sfv = e4m3_value(sfb);
-            if (sfv > 0.0f) {
-                const float inv = __fdiv_rn(gs, sfv);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t byte = e2m1x2_rn_satfinite(__fmul_rn(v[2 * i], inv), __fmul_rn(v[2 * i + 1], inv));
-                    packed[i >> 2] |= byte << ((i & 3) * 8);
-                }
-            }
-            *reinterpret_cast<uint2*>(codes + r * (k / 2) + c * 8) = make_uint2(packed[0], packed[1]);
+            uint2 packed;
+            sfb = quantize_block(__ldg(src), __ldg(src + 1), gs, packed);
+            *reinterpret_cast<uint2*>(codes + r * (k / 2) + c * 8) = packed;
         }
         // four consecutive blocks of a row: one 4-byte store into the swizzled scale atom
         const uint32_t b1 = __shfl_down_sync(0xffffffffu, sfb, 1);
