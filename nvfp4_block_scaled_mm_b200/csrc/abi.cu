@@ -515,8 +515,17 @@ nvfp4lora_status launch_fold(const uint16_t* lora_b, const float* lora_scale, co
     const int64_t groups = N * r / 8;
     const int64_t want = (groups + kFoldThreads - 1) / kFoldThreads;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)info->sms * 8));
-    fold_kernel<<<grid, kFoldThreads, 0, stream>>>(lora_b, lora_scale, alpha, b_folded, ratio, groups);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kFoldThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fold_kernel, lora_b, lora_scale, alpha, b_folded, ratio, groups);
     if (e != cudaSuccess) return cuda_fail(e, "fold launch");
     return NVFP4LORA_OK;
 }

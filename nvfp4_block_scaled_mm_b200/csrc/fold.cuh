@@ -30,7 +30,11 @@ constexpr int kFoldThreads = 256;
 __global__ void __launch_bounds__(kFoldThreads)
 fold_kernel(const uint16_t* lora_b, const float* lora_scale, const float* alpha,
             uint16_t* b_folded, float* ratio_out, int64_t groups) {
-    // Let a dependent GEMM begin its prologue; it still waits for this grid before reading.
+    // Launched with programmatic dependent launch: the CTAs start while the previous kernel on
+    // the stream (typically the GEMM that reads b_folded) finishes, and wait for it here before
+    // any read or write.  A dependent GEMM may begin its prologue at once; it still waits for
+    // this grid before reading.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const float ratio = __fdiv_rn(*lora_scale, *alpha);
     if (blockIdx.x == 0 && threadIdx.x == 0) *ratio_out = ratio;
