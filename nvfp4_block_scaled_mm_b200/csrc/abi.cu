@@ -475,11 +475,13 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     return NVFP4LORA_OK;
 }
 
-// The SM-pair kernel measured level with the single-SM one where both run the same number of
-// waves, and worse where its 256-row tiles add a wave (or at M = 256): it is used from M = 512 on
-// when its wave count over the SM pairs is no larger than the single-SM kernel's over the SMs.
+// The SM-pair kernel measured faster than the single-SM one on every shape with M >= 128 where both
+// run the same number of waves (2-6 % at M = 128..384, N = 14336; 20-30 % at M >= 2048 since it
+// stages scales with register stores and halves each SM's B traffic), and slower where its 256-row
+// tiles add a wave (4736 x 1024 x 8192: 31.8 against 20.9 us).  It is used from M = 128 on when its
+// wave count over the SM pairs is no larger than the single-SM kernel's over the SMs.
 bool use_pair_kernel(int64_t M, int64_t N) {
-    if (M < 512) return false;
+    if (M < 128) return false;
     int dev = 0;
     DeviceInfo* info = nullptr;
     if (device_info(&dev, &info) != NVFP4LORA_OK) return false;
