@@ -130,20 +130,27 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def source_hash():
+def source_hash(kernel="gemm"):
+    """Hash of the sources a kernel's recorded ncu figures depend on: its own kernel files and the
+    host launcher (abi.cu).  The GEMM kernels depend on every source but the quantizer's."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "nvfp4_block_scaled_mm_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    files = sorted(os.listdir(d))
+    if kernel == "quantize":
+        files = ["abi.cu", "quantize.cuh"]
+    else:
+        files = [f for f in files if f != "quantize.cuh"]
+    for f in files:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per launch of the GEMM kernel from the committed ncu summary, if it was
-    taken on the current kernel sources (else None)."""
-    path = os.path.join(PROFILES, f"gemm_{workload}_traffic.md")
+def recorded_traffic(workload, kernel="gemm"):
+    """DRAM bytes per launch of the workload's dominant kernel (`gemm` or `quantize`) from the
+    committed ncu summary, if it was taken on the current kernel sources (else None)."""
+    path = os.path.join(PROFILES, f"{kernel}_{workload}_traffic.md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -152,7 +159,7 @@ def recorded_traffic(workload):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_sha") != source_hash():
+    if vals.get("source_sha") != source_hash(kernel):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -476,6 +483,9 @@ def run_quant(args, rank, world, device):
     if world > 1:
         ms = max_over_ranks(ms, device)
     value = nbytes / (ms * 1e-3) / 1e9
+    e2e = run_quant_e2e(L, x, gs, device, stream, min(steps, 50))
+    if world > 1:
+        e2e["ms_step"] = max_over_ranks(e2e["ms_step"], device)
     peaks, peak_src = measured_peaks()
     line = {
         "metric": METRIC, "value": whole_job(value, world), "unit": "GB/s", "n_gpus": world, "steps": steps,
@@ -486,11 +496,14 @@ def run_quant(args, rank, world, device):
                    "l2_defeat": "inputs rotate through copies totalling >= 3x L2",
                    "timing": "CUDA graph of K back-to-back calls, CUDA events on the launching stream"},
         "roofline": {"bound": "hbm", "achieved": value, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": value / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}", "traffic": None,
-                     "algorithmic_bytes_per_launch": nbytes},
+                     "frac": value / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}",
+                     "traffic": recorded_traffic("quant", kernel="quantize"), "algorithmic_bytes_per_launch": nbytes},
         "clocks": clk.summary(),
-        "e2e": {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
-                "note": "not measured for the quantizer; the end-to-end figures are the GEMM lines'"},
+        "e2e": {"value": whole_job(nbytes / (e2e["ms_step"] * 1e-3) / 1e9, world), "unit": "GB/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "ms_per_step": e2e["ms_step"], "steps": e2e["steps"],
+                "method": "fp4_quantize on device buffers filled from pinned host memory each step, codes and "
+                          "scales copied back; two step slots, copies and calls on three streams, one CUDA graph"},
         "gpu_launches": steps,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -511,6 +524,75 @@ def run_quant(args, rank, world, device):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_quant_e2e(L, x, gs, device, stream, steps):
+    """The quantizer end to end through fp4_quantize with host buffers: each step copies the bf16
+    activations host -> device from pinned memory, quantizes, and copies the codes and scales back
+    to pinned memory.  Two step slots alternate over three streams ordered by events (as in the
+    GEMM's end-to-end run), replayed from one CUDA graph."""
+    slots = 2
+    rows, K = x.shape
+    n_sf = (rows + 127) // 128 * 128 * (K // 16)
+    host_x = [x.pin_memory() for _ in range(slots)]
+    dev_x = [torch.empty_like(x, device=device) for _ in range(slots)]
+    dev_c = [torch.empty((rows, K // 2), dtype=torch.uint8, device=device) for _ in range(slots)]
+    dev_s = [torch.empty(n_sf, dtype=torch.uint8, device=device) for _ in range(slots)]
+    host_c = [torch.empty((rows, K // 2), dtype=torch.uint8).pin_memory() for _ in range(slots)]
+    host_s = [torch.empty(n_sf, dtype=torch.uint8).pin_memory() for _ in range(slots)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    n_ev = steps + 8
+    ev_in = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_call = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_out = [torch.cuda.Event() for _ in range(n_ev)]
+
+    def one(i, first):
+        k = i % slots
+        with torch.cuda.stream(s_in):
+            if i - first >= slots:
+                s_in.wait_event(ev_call[i - slots])
+            dev_x[k].copy_(host_x[k], non_blocking=True)
+            ev_in[i].record(s_in)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[i])
+            if i - first >= slots:
+                stream.wait_event(ev_out[i - slots])
+            L.fp4_quantize(dev_x[k], gs, codes=dev_c[k], scales=dev_s[k])
+            ev_call[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_call[i])
+            host_c[k].copy_(dev_c[k], non_blocking=True)
+            host_s[k].copy_(dev_s[k], non_blocking=True)
+            ev_out[i].record(s_out)
+
+    for i in range(4):
+        one(i, 0)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        s_in.wait_event(fork)
+        s_out.wait_event(fork)
+        for i in range(steps):
+            one(i + 4, 4)
+        for st_ in (s_in, s_out):
+            join = torch.cuda.Event()
+            join.record(st_)
+            stream.wait_event(join)
+    g.replay()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    L.nvfp4lora_device_status(stream)
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    return dict(ms_step=ms, steps=steps, h2d=x.numel() * 2, d2h=rows * K // 2 + n_sf)
 
 
 def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):

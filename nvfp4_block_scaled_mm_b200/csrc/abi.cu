@@ -130,9 +130,17 @@ nvfp4lora_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
 
 // 2-D row-major tensor [rows, cols] of `esize`-byte elements, read in boxes of
 // box_cols x box_rows with the 128-byte swizzle; out-of-range elements read as zero.
+// The LoRA operands d [M, r] and lora_b / b_folded [N, r] of the tiled kernels are read with no L2
+// promotion.  Their boxes are 64 columns wide and zero-filled past r; where r is not a multiple of
+// 16 a row's in-bounds part ends inside a 32-byte sector, and with 256-byte promotion those loads
+// arrived late enough to stall the tile's end: raw path, M = 256, N = 14336, K = 4096, r = 8 ran
+// 18.3 us on the SM-pair kernel with promotion and 16.9 without (r = 16: 14.9 either way).
+constexpr CUtensorMapL2promotion kLoraPromotion = CU_TENSOR_MAP_L2_PROMOTION_NONE;
+
 nvfp4lora_status encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int esize,
                            uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
-                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B,
+                           CUtensorMapL2promotion promotion = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
     nvfp4lora_status st = get_encoder(&enc);
     if (st != NVFP4LORA_OK) return st;
@@ -141,8 +149,7 @@ nvfp4lora_status encode_2d(CUtensorMap* map, const void* base, CUtensorMapDataTy
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promotion, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(NVFP4LORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
     return NVFP4LORA_OK;
 }
@@ -252,8 +259,8 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, kTileM)) != NVFP4LORA_OK) return st;
     if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, kTileN)) != NVFP4LORA_OK) return st;
     if (MODE != Mode::Off) {
-        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, kTileM)) != NVFP4LORA_OK) return st;
-        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, kTileN)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B, kLoraPromotion)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, kTileN, CU_TENSOR_MAP_SWIZZLE_128B, kLoraPromotion)) != NVFP4LORA_OK) return st;
     }
     // rows of out 16-byte aligned: the epilogue writes 32 x 32 bf16 boxes with TMA stores
     const bool vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16)));
@@ -422,10 +429,10 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
     if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) != NVFP4LORA_OK) return st;
     if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) != NVFP4LORA_OK) return st;
     if (MODE != Mode::Off) {
-        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, kLoraPromotion)) != NVFP4LORA_OK) return st;
         // raw: per N-half, 64 of each CTA's 128 lora_b rows; prepared: all 128
         const int lb_rows = (MODE == Mode::Raw) ? 64 : 128;
-        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, lb_rows)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, N, 64, lb_rows, CU_TENSOR_MAP_SWIZZLE_128B, kLoraPromotion)) != NVFP4LORA_OK) return st;
     }
     const bool vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16)));
     if (vec_out &&
@@ -480,8 +487,14 @@ nvfp4lora_status launch_gemm_pair(const uint8_t* a, const uint8_t* b, const uint
 // stages scales with register stores and halves each SM's B traffic), and slower where its 256-row
 // tiles add a wave (4736 x 1024 x 8192: 31.8 against 20.9 us).  It is used from M = 128 on when its
 // wave count over the SM pairs is no larger than the single-SM kernel's over the SMs.
-bool use_pair_kernel(int64_t M, int64_t N) {
+//
+// One exception, measured on the raw path with a rank below 32 that is not a multiple of 16 (the
+// narrow-row LoRA loads above) at M <= 256: 256 x 14336 x 4096, r = 8 ran 15.5 us on the single-SM
+// kernel against 16.9 on the pair kernel (128 rows: 15.2 against 16.1), so those calls stay on the
+// single-SM kernel.
+bool use_pair_kernel(int64_t M, int64_t N, bool raw, int64_t r) {
     if (M < 128) return false;
+    if (raw && r % 16 != 0 && r < 32 && M <= 256) return false;
     int dev = 0;
     DeviceInfo* info = nullptr;
     if (device_info(&dev, &info) != NVFP4LORA_OK) return false;
@@ -499,7 +512,7 @@ nvfp4lora_status launch(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf,
                         const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
     if (M <= kDecodeMaxM)
         return launch_decode<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
-    if (use_pair_kernel(M, N))
+    if (use_pair_kernel(M, N, MODE == Mode::Raw, r))
         return launch_gemm_pair<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
     return launch_gemm<MODE>(a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M, N, K, stream);
 }
