@@ -330,15 +330,15 @@ def run_ours(args, rank, world, device):
 
     # end to end through the public API with host buffers: per step, the activation-side
     # inputs (a, a_sf, d) go host -> device and the output comes back device -> host.
-    e2e = run_e2e(L, p, sets[0], alpha, s, out, c, device, stream, min(K_steps, 2000), prepared,
-                  adapters[0] if prepared else None)
+    e2e = run_e2e(L, p, sets, alpha, s, out, c, device, stream, min(K_steps, 2000), prepared,
+                  adapters if prepared else None)
 
     return dict(c=c, ms=ms, ms_step=ms_step, K=K_steps, W=max(W, 3), nbytes=nbytes, flops=flops,
                 lora_flops=lora_flops, copies=copies, clocks=clk.summary(), e2e=e2e,
                 launches=K_steps * launches_per_step, in_bytes=in_bytes, l2=l2, p=p, overhead=overhead)
 
 
-def cfg4_point(L, M, r, device, stream, l2):
+def cfg4_point(L, M, r, device, stream, l2, e2e=False):
     """One point of the adapter-switch sweep: N=14336, K=4096, 8 adapters switched every call.
     Times, each as a CUDA graph of back-to-back calls: the raw path with a different adapter's
     pointers per call; the prepared path refolding the next adapter inside the graph (fold +
@@ -391,6 +391,15 @@ def cfg4_point(L, M, r, device, stream, l2):
         ms = time_graph(fn, n, stream, device)
         res[name] = {"us_per_call": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9, "tflops": flops / (ms * 1e-3) / 1e12}
     L.nvfp4lora_device_status(stream)
+    if e2e:
+        # the raw swap end to end: a, a_sf and d from pinned host memory, out back, weights and
+        # adapters rotating as in the device-timed graph
+        sets = [dict(b=weights[i % copies][0], b_sf=weights[i % copies][1], lora_b=adps[i % na][0],
+                     s=adps[i % na][1], bias=None) for i in range(max(copies, na))]
+        e = run_e2e(L, p, sets, alpha, None, out, c, device, stream, min(n, 2000), False, None)
+        res["e2e"] = {"value": nbytes / (e["ms_step"] * 1e-3) / 1e9, "unit": "GB/s",
+                      "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                      "ms_per_step": e["ms_step"], "steps": e["steps"]}
     return res
 
 
@@ -405,7 +414,7 @@ def run_cfg4(args, rank, world, device):
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         for M in CFG4["Ms"]:
             for r in CFG4["rs"]:
-                sweep.append(cfg4_point(L, M, r, device, stream, l2))
+                sweep.append(cfg4_point(L, M, r, device, stream, l2, e2e=not sweep))
                 torch.cuda.empty_cache()
     head = sweep[0]
     ms = head["raw_swap"]["us_per_call"] * 1e-3
@@ -426,8 +435,12 @@ def run_cfg4(args, rank, world, device):
         "roofline": {"bound": "hbm", "achieved": value, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": value / peaks["hbm_gbs"], "peak_source": f"hbm_gbs of {peak_src}", "traffic": None},
         "clocks": clk.summary(),
-        "e2e": {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
-                "note": "not measured for the sweep; the end-to-end figure is the cfg1 line's"},
+        "e2e": {"value": whole_job(head["e2e"]["value"], world), "unit": "GB/s",
+                "h2d_bytes_per_step": head["e2e"]["h2d_bytes_per_step"],
+                "d2h_bytes_per_step": head["e2e"]["d2h_bytes_per_step"],
+                "ms_per_step": head["e2e"]["ms_per_step"], "steps": head["e2e"]["steps"],
+                "method": "raw swap at M=1 r=8 through mm_nvfp4_lora: a, a_sf, d copied from pinned host memory "
+                          "and out copied back every step; two step slots on three streams, one CUDA graph"},
         # this library's kernels per call: raw 1; refold + GEMM 2 (the copy_ kernels are PyTorch's)
         "gpu_launches": sum(pt["calls"] * k for pt in sweep for k in (1, 2, 2)),
         "sweep": sweep,
@@ -595,14 +608,16 @@ def run_quant_e2e(L, x, gs, device, stream, steps):
     return dict(ms_step=ms, steps=steps, h2d=x.numel() * 2, d2h=rows * K // 2 + n_sf)
 
 
-def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
+def run_e2e(L, p, sets, alpha, s, out, c, device, stream, steps, prepared, adps):
     """End to end through the public API with host buffers.  Every step copies its activation-side
     inputs (a, a_sf, d) host -> device from pinned memory, makes the call, and copies out back to
     pinned host memory.  a's, a_sf's and d's bytes sit in one pinned staging buffer (one copy per
-    step).  Steps are pipelined the way a serving loop would run them: two step slots alternate,
-    and the host -> device copies, the calls and the device -> host copies run on three streams
-    ordered by events, so one step's copies overlap its neighbours' calls.  The timed steps are
-    replayed from one CUDA graph."""
+    step).  The resident weights (b, b_sf, lora_b or the prepared adapter, bias) rotate through
+    the same device copies as the device-timed loop, so they are read from HBM, not L2.  Steps are
+    pipelined the way a serving loop would run them: two step slots alternate, and the host ->
+    device copies, the calls and the device -> host copies run on three streams ordered by
+    events, so one step's copies overlap its neighbours' calls.  The timed steps are replayed
+    from one CUDA graph."""
     def region(nbytes):
         return (nbytes + 255) // 256 * 256
     na, nsf, nd = p.a.numel(), p.a_sf.numel(), p.d.numel() * 2
@@ -649,12 +664,13 @@ def run_e2e(L, p, st, alpha, s, out, c, device, stream, steps, prepared, adp):
                 if i - first >= slots:
                     stream.wait_event(ev_out[i - slots])    # the slot's previous output has been copied out
             a_d, a_sf_d, d_d = views[k]
+            st = sets[i % len(sets)]
             if prepared:
-                L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, lora_adapter=adp, bias=st["bias"],
-                                out=outs[k])
+                L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, lora_adapter=adps[i % len(adps)],
+                                bias=st["bias"], out=outs[k])
             else:
-                L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, st["lora_b"], s, bias=st["bias"],
-                                out=outs[k])
+                L.mm_nvfp4_lora(a_d, st["b"], a_sf_d, st["b_sf"], alpha, d_d, st["lora_b"], st.get("s", s),
+                                bias=st["bias"], out=outs[k])
             if pipelined:
                 ev_call[i].record(stream)
         with torch.cuda.stream(s_out):
@@ -905,7 +921,7 @@ def main():
         "config": config_block(args, c), "roofline": roof, "clocks": res["clocks"],
         "e2e": {"value": whole_job(e2e_val, world), "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"],
-                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; two step slots pipelined over three streams; the steps captured in one CUDA graph; weights resident"},
+                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; two step slots pipelined over three streams; the steps captured in one CUDA graph; weights resident in HBM, rotating through the same copies as the device-timed loop"},
         "gpu_launches": res["launches"],
         "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
         "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],

@@ -95,3 +95,23 @@ def test_quantize_then_gemm_matches_oracle_composition():
     ref = xa.double() @ xb.double().T
     rel = torch.linalg.norm(torch.from_numpy(got) - ref) / torch.linalg.norm(ref)
     assert rel < 0.2
+
+
+def test_quantize_full_size_workload_sampled_row_blocks():
+    """The benchmarked workload (bf16 [8192, 8192] activations, the A operand of the
+    8192 x 28672 x 8192 GEMM, with the quantizer bench's generator and seed) through the same
+    launch; the oracle checks the
+    first, a middle and the last 128-row block bit for bit (rows are independent, and a 128-row
+    block's scale bytes are one contiguous run of the swizzled layout)."""
+    rows, k = 8192, 8192
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(rows, k, generator=g) * 2.0).to(torch.bfloat16)
+    gs = 448.0 * 6.0 / x.float().abs().max().item()
+    codes, scales = _run(x, gs)
+    nb = k // 16
+    block_bytes = 128 * nb
+    for rb in (0, rows // 256, rows // 128 - 1):
+        xb = x[rb * 128:(rb + 1) * 128]
+        want_codes, want_scales = O.quantize_nvfp4(_bf16_bits(xb), gs)
+        np.testing.assert_array_equal(codes[rb * 128:(rb + 1) * 128], want_codes)
+        np.testing.assert_array_equal(scales[rb * block_bytes:(rb + 1) * block_bytes], want_scales)
