@@ -440,7 +440,7 @@ def run_cfg4(args, rank, world, device):
                 "d2h_bytes_per_step": head["e2e"]["d2h_bytes_per_step"],
                 "ms_per_step": head["e2e"]["ms_per_step"], "steps": head["e2e"]["steps"],
                 "method": "raw swap at M=1 r=8 through mm_nvfp4_lora: a, a_sf, d copied from pinned host memory "
-                          "and out copied back every step; two step slots on three streams, one CUDA graph"},
+                          "and out copied back every step; four step slots on three streams, one CUDA graph"},
         # this library's kernels per call: raw 1; refold + GEMM 2 (the copy_ kernels are PyTorch's)
         "gpu_launches": sum(pt["calls"] * k for pt in sweep for k in (1, 2, 2)),
         "sweep": sweep,
@@ -608,22 +608,25 @@ def run_quant_e2e(L, x, gs, device, stream, steps):
     return dict(ms_step=ms, steps=steps, h2d=x.numel() * 2, d2h=rows * K // 2 + n_sf)
 
 
-def run_e2e(L, p, sets, alpha, s, out, c, device, stream, steps, prepared, adps):
+def run_e2e(L, p, sets, alpha, s, out, c, device, stream, steps, prepared, adps, slots=None):
     """End to end through the public API with host buffers.  Every step copies its activation-side
     inputs (a, a_sf, d) host -> device from pinned memory, makes the call, and copies out back to
     pinned host memory.  a's, a_sf's and d's bytes sit in one pinned staging buffer (one copy per
     step).  The resident weights (b, b_sf, lora_b or the prepared adapter, bias) rotate through
     the same device copies as the device-timed loop, so they are read from HBM, not L2.  Steps are
-    pipelined the way a serving loop would run them: two step slots alternate, and the host ->
-    device copies, the calls and the device -> host copies run on three streams ordered by
-    events, so one step's copies overlap its neighbours' calls.  The timed steps are replayed
+    pipelined the way a serving loop would run them: step slots (four, or two for a
+    large output) rotate, and the host -> device copies, the calls and the device -> host copies
+    run on three streams ordered by events, so one step's copies overlap its neighbours' calls.  The timed steps are replayed
     from one CUDA graph."""
     def region(nbytes):
         return (nbytes + 255) // 256 * 256
     na, nsf, nd = p.a.numel(), p.a_sf.numel(), p.d.numel() * 2
     oa, osf, od = 0, region(na), region(na) + region(nsf)
     total = od + region(nd)
-    slots = 2
+    # four steps in flight where a step's output is small (the copies are latency-bound: cfg1
+    # runs 1231 GB/s with four slots against 1013 with two, and eight add nothing); two where
+    # it is large, to bound the pinned host memory (cfg3: 470 MB per slot)
+    slots = slots or (4 if out.numel() * 2 <= (64 << 20) else 2)
     host_in, dev_in, views = [], [], []
     for _ in range(slots):
         h = torch.empty(total, dtype=torch.uint8).pin_memory()
@@ -921,7 +924,7 @@ def main():
         "config": config_block(args, c), "roofline": roof, "clocks": res["clocks"],
         "e2e": {"value": whole_job(e2e_val, world), "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"],
-                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; two step slots pipelined over three streams; the steps captured in one CUDA graph; weights resident in HBM, rotating through the same copies as the device-timed loop"},
+                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; step slots (4, or 2 for outputs over 64 MB) pipelined over three streams; the steps captured in one CUDA graph; weights resident in HBM, rotating through the same copies as the device-timed loop"},
         "gpu_launches": res["launches"],
         "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
         "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],
