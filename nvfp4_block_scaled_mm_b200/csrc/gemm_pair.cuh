@@ -265,13 +265,16 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                 // ring items: base stages; raw: the previous tile's LoRA half 1 before base stage
                 // kRawHalf1At (or after the base stages), this tile's half 0 after them; prepared:
                 // the LoRA chunks after the base stages
+                // (two segments around the half-1 point: no check for it in the per-stage loop)
                 const int h1_at = min(kRawHalf1At, args.k_stages);
-                for (int it = 0; ok && it <= args.k_stages; ++it) {
-                    if (MODE == Mode::Raw && pend && it == h1_at) {
+                int it = 0;
+                for (int seg = 0; ok && seg < 2; ++seg) {
+                    const int it_end = seg == 0 ? h1_at : args.k_stages;
+                    for (; ok && it < it_end; ++it) ok = emit_base(it, row_a, row_b);
+                    if (ok && seg == 0 && MODE == Mode::Raw && pend) {
                         for (int c = 0; ok && c < lora_chunks_if_on; ++c) ok = emit_half(c, 1, prev_m, prev_n);
                         pend = false;
                     }
-                    if (ok && it < args.k_stages) ok = emit_base(it, row_a, row_b);
                 }
                 if (ok && lora_on) {
                     if (MODE == Mode::Raw) {
@@ -375,27 +378,32 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                 // both CTAs' epilogues have read the previous tile's accumulator
                 if (!mbar_wait_cluster(acc_empty, (i & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int it = 0; ok && it < args.k_stages; ++it) {
-                    if (MODE == Mode::Raw && pend && it == h1_at && !finish_pending()) { ok = false; break; }
-                    // both CTAs staged this slot's scales, and both CTAs' code tiles landed
-                    if (!mbar_wait_cluster(&sf_ready[slot], slot_use & 1u, abort_flag)) { ok = false; break; }
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + L::A_OFF + stage * L::A_BYTES);
-                    const uint32_t b_addr = smem_u32(smem + L::B_OFF + stage * L::B_BYTES);
-                    const uint32_t sfa_t = tmem + T::SF0 + slot * T::SLOT_COLS;
-                    const uint32_t sfb_t = sfa_t + T::SFA_COLS;
+                // the base stages, in two segments around the half-1 point so that the issue loop
+                // itself carries no check for it (one there cost about 4 % in the raw kernel)
+                int it = 0;
+                for (int seg = 0; ok && seg < 2; ++seg) {
+                    const int it_end = seg == 0 ? h1_at : args.k_stages;
+                    for (; it < it_end; ++it) {
+                        // both CTAs staged this slot's scales, and both CTAs' code tiles landed
+                        if (!mbar_wait_cluster(&sf_ready[slot], slot_use & 1u, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a_addr = smem_u32(smem + L::A_OFF + stage * L::A_BYTES);
+                        const uint32_t b_addr = smem_u32(smem + L::B_OFF + stage * L::B_BYTES);
+                        const uint32_t sfa_t = tmem + T::SF0 + slot * T::SLOT_COLS;
+                        const uint32_t sfb_t = sfa_t + T::SFA_COLS;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tc_mma_nvf4_pair(tmem + T::ACC, sdesc_sw128(a_addr + j * 32), sdesc_sw128(b_addr + j * 32),
-                                         IDESC_F4, sfa_t + 4 * j, sfb_t + 8 * j, (it > 0 || j > 0) ? 1u : 0u);
-                    tc_commit_pair_multicast(&empty[stage], kBoth);
-                    tc_commit_pair_multicast(&slot_free[slot], kBoth);
-                    if (++slot == T::NSF) { slot = 0; ++slot_use; }
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                        for (int j = 0; j < 4; ++j)
+                            tc_mma_nvf4_pair(tmem + T::ACC, sdesc_sw128(a_addr + j * 32), sdesc_sw128(b_addr + j * 32),
+                                             IDESC_F4, sfa_t + 4 * j, sfb_t + 8 * j, (it > 0 || j > 0) ? 1u : 0u);
+                        tc_commit_pair_multicast(&empty[stage], kBoth);
+                        tc_commit_pair_multicast(&slot_free[slot], kBoth);
+                        if (++slot == T::NSF) { slot = 0; ++slot_use; }
+                        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    }
+                    if (ok && seg == 0 && MODE == Mode::Raw && pend && !finish_pending()) ok = false;
                 }
                 if (!ok) break;
-                if (MODE == Mode::Raw && pend && !finish_pending()) { ok = false; break; }   // k_stages <= h1_at
                 if (lora_on && MODE == Mode::Prepared) {
                     // the folded LoRA term into the same accumulator, after the base product
                     for (int c = 0; ok && c < lora_chunks_if_on; ++c) {
@@ -520,13 +528,15 @@ nvfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                 // once lacc_full says so, after the h = 0 warps of both CTAs have released half 0
                 if (h == 1 && !__all_sync(kAll, mbar_wait(lacc_full, i & 1, abort_flag))) break;
                 tc_fence_after();
+                // 16 columns at a time: with the 128 held values this keeps the epilogue within
+                // its registers (32-column reads spilled)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t lv[32];
-                    tmem_load_32(tmem + lane_off + T::LACC + c * 32, lv);
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t lv[16];
+                    tmem_load_16(tmem + lane_off + T::LACC + c * 16, lv);
                     tmem_load_wait();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) v[c * 32 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 32 + k]);
+                    for (int k = 0; k < 16; ++k) v[c * 16 + k] = __fmaf_rn(lora_s, __uint_as_float(lv[k]), v[c * 16 + k]);
                 }
                 tc_fence_before();
                 if (rank == 0) mbar_arrive(lacc_empty);
