@@ -20,7 +20,7 @@ It restates, slowly and in float64, what the pages define:
 * the quantizer the mm_nvfp4_lora page names as the producer of a / a_sf (``fp4_quantize``),
   by the reading given at :func:`quantize_nvfp4`.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * nibble order: element ``2j`` of a row is the LOW nibble of byte ``j``.  The GEMM
   result does not depend on it (both nibbles of a byte sit in the same 16-block and
@@ -322,7 +322,7 @@ def eager_prepare_check(lora_scale: float, alpha: float) -> None:
 # says the operands come "in the 128x4 swizzled layout produced by fp4_quantize()"; Parameters:
 # alpha is "alpha_base / (a_global_scale * b_global_scale)", so dequant(codes, scales) carries
 # a per-tensor global scale).  The pages name the quantizer but not its rule.  The reading
-# taken (listed in the design doc), each step in float32 as the kernel computes it:
+# taken, each step in float32 as the kernel computes it:
 #   per 16-element block along K:  amax = max |x|                (x: bf16, exact in float32)
 #   sf    = E4M3(rne, saturate to 448)( (amax * gs) / 6 )         (6 = largest E2M1 value)
 #   inv   = gs / value(sf)               (sf == 0: every code of the block is +0)
