@@ -466,6 +466,14 @@ def run_cfg4(args, rank, world, device):
         "gpu_launches": sum(pt["calls"] * k for pt in sweep for k in (1, 2, 2)),
         "sweep": sweep,
     }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle on the headline point (M=1, r=8, raw path), as the reference arm times it
+        from workloads import make_problem
+        c = describe("cfg4")
+        p = make_problem(c["M"], c["N"], c["K"], c["r"], c["seed"], alpha=c["alpha"],
+                         lora_scale=c["lora_scale"], bias=c["bias"])
+        nb, fl, _ = algorithmic(c)
+        line["cpu_baseline"] = cpu_baseline(p, c, nb, fl)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
