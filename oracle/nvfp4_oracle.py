@@ -228,56 +228,74 @@ def base_product_rows_cols(a, b, a_sf, b_sf, K: int, rows, cols) -> np.ndarray:
     return dequant_rows(a, a_sf, K, rows) @ dequant_rows(b, b_sf, K, cols).T
 
 
-def lora_term(d_bits, lb_bits, M: int, N: int, r: int) -> np.ndarray:
-    """``d @ lora_b^T`` in float64 (bf16 x bf16 products are exact in float64)."""
-    d = bf16_bits_to_f64(np.asarray(d_bits).reshape(M, r))
-    lb = bf16_bits_to_f64(np.asarray(lb_bits).reshape(N, r))
+def _pick(idx, count: int) -> np.ndarray:
+    """The selected output rows (or columns): all of them when ``idx`` is None."""
+    return np.arange(count) if idx is None else np.asarray(idx, dtype=np.int64)
+
+
+def lora_term(d_bits, lb_bits, M: int, N: int, r: int, rows=None, cols=None) -> np.ndarray:
+    """``d @ lora_b^T`` in float64 (bf16 x bf16 products are exact in float64), restricted to
+    the output ``rows`` x ``cols`` when given."""
+    d = bf16_bits_to_f64(np.asarray(d_bits).reshape(M, r))[_pick(rows, M)]
+    lb = bf16_bits_to_f64(np.asarray(lb_bits).reshape(N, r))[_pick(cols, N)]
     return d @ lb.T
 
 
-def _bias_row(bias_bits, N: int):
+def _bias_row(bias_bits, N: int, cols=None):
     if bias_bits is None:
         return 0.0
-    return bf16_bits_to_f64(np.asarray(bias_bits).reshape(N))[None, :]
+    return bf16_bits_to_f64(np.asarray(bias_bits).reshape(N))[_pick(cols, N)][None, :]
 
+
+def _base(a, b, a_sf, b_sf, M: int, N: int, K: int, rows, cols) -> np.ndarray:
+    if rows is None and cols is None:
+        return base_product(a, b, a_sf, b_sf, M, N, K)
+    return base_product_rows_cols(a, b, a_sf, b_sf, K, _pick(rows, M), _pick(cols, N))
+
+
+# The three call forms below take optional ``rows`` / ``cols`` (index arrays): the same
+# definition evaluated on the selected outputs only, for sampled checks at full sizes.  A
+# caller-supplied ``base`` must already cover exactly those outputs.
 
 def mm_raw(a, b, a_sf, b_sf, alpha: float, d_bits, lb_bits, lora_scale, bias_bits,
-           M: int, N: int, K: int, r: int, base: np.ndarray | None = None) -> np.ndarray:
+           M: int, N: int, K: int, r: int, base: np.ndarray | None = None,
+           rows=None, cols=None) -> np.ndarray:
     """Raw path ("Raw path" bullet): ``alpha*base + s*(d @ lora_b^T) [+ bias]``, float64.
 
     ``lora_scale`` None or equal to zero is the zero-adapter call (Parameters:
     lora_scale): the LoRA term is not evaluated at all.
     """
     if base is None:
-        base = base_product(a, b, a_sf, b_sf, M, N, K)
+        base = _base(a, b, a_sf, b_sf, M, N, K, rows, cols)
     y = np.float64(alpha) * base
     if lora_scale is not None and float(lora_scale) != 0.0:
-        y = y + np.float64(lora_scale) * lora_term(d_bits, lb_bits, M, N, r)
-    return y + _bias_row(bias_bits, N)
+        y = y + np.float64(lora_scale) * lora_term(d_bits, lb_bits, M, N, r, rows, cols)
+    return y + _bias_row(bias_bits, N, cols)
 
 
 def mm_prepared(a, b, a_sf, b_sf, alpha: float, d_bits, b_folded_bits, ratio, bias_bits,
-                M: int, N: int, K: int, r: int, base: np.ndarray | None = None) -> np.ndarray:
+                M: int, N: int, K: int, r: int, base: np.ndarray | None = None,
+                rows=None, cols=None) -> np.ndarray:
     """Prepared path ("Prepared path" bullet): base first, LoRA with ``b_folded`` into the
     same accumulator, alpha applied once: ``alpha*(base + d @ b_folded^T) [+ bias]``.
 
     ``ratio`` is the fold's ``lora_scale / alpha``; a zero ratio is the zero adapter
-    (Parameters: lora_adapter -- "lora_scale == 0 produces the adapter-off output").
+    (Parameters: lora_adapter -- a zero lora_scale gives the adapter-off output).
     """
     if base is None:
-        base = base_product(a, b, a_sf, b_sf, M, N, K)
+        base = _base(a, b, a_sf, b_sf, M, N, K, rows, cols)
     acc = base
     if float(ratio) != 0.0:
-        acc = acc + lora_term(d_bits, b_folded_bits, M, N, r)
-    return np.float64(alpha) * acc + _bias_row(bias_bits, N)
+        acc = acc + lora_term(d_bits, b_folded_bits, M, N, r, rows, cols)
+    return np.float64(alpha) * acc + _bias_row(bias_bits, N, cols)
 
 
 def mm_off(a, b, a_sf, b_sf, alpha: float, bias_bits, M: int, N: int, K: int,
-           base: np.ndarray | None = None) -> np.ndarray:
+           base: np.ndarray | None = None, rows=None, cols=None) -> np.ndarray:
     """Adapter-off call (neither form): ``alpha*base [+ bias]``."""
     if base is None:
-        base = base_product(a, b, a_sf, b_sf, M, N, K)
-    return np.float64(alpha) * base + _bias_row(bias_bits, N)
+        base = _base(a, b, a_sf, b_sf, M, N, K, rows, cols)
+    return np.float64(alpha) * base + _bias_row(bias_bits, N, cols)
 
 
 def round_output(y: np.ndarray) -> np.ndarray:

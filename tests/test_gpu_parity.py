@@ -212,6 +212,49 @@ def test_off_parity(M, N, K):
     check_close(out, O.mm_off(h["a"], h["b"], h["a_sf"], h["b_sf"], p.alpha, h["bias"], M, N, K), what="off")
 
 
+# ---------------------------------------------------------------------------------------
+# the whole finite UE4M3 range (subnormal scales 0x01..0x07 up to 448 = 0x7E) on every kernel and
+# every path (flashinfer.gemm.mm_nvfp4_lora: the paragraph after the formula and Parameters: a_sf,
+# b_sf -- UE4M3 block scales of 16 along K)
+# ---------------------------------------------------------------------------------------
+
+# (kernel the shape dispatches to, M, N, K, r): M <= 16 decode with 16 token columns, 17..32 decode
+# with 32, 33..127 the single-SM tiled kernel, 256 rows here the SM-pair kernel (r >= 32 keeps the
+# raw path on it); N = 520 leaves a ragged last tile on each
+RANGE_SHAPES = [("decode16", 16, 520, 1024, 40), ("decode32", 20, 520, 512, 40),
+                ("single_sm", 64, 520, 1024, 40), ("sm_pair", 256, 520, 1024, 40)]
+SCALE_RANGES = [("full", (0x01, 0x7E), (0x01, 0x7E)),
+                ("a_subnormal", (0x01, 0x07), (0x01, 0x7E)),
+                ("a_large_b_subnormal", (0x70, 0x7E), (0x01, 0x07))]
+
+
+@pytest.mark.parametrize("kernel,M,N,K,r", RANGE_SHAPES)
+@pytest.mark.parametrize("name,ra,rb", SCALE_RANGES)
+def test_full_ue4m3_scale_range_every_kernel_and_path(kernel, M, N, K, r, name, ra, rb):
+    """Scale bytes drawn over whole UE4M3 sub-ranges; alpha is the power of two that brings the
+    base product to unit RMS, so the LoRA term stays comparable and both are checked."""
+    p = make_problem(M, N, K, r, seed=M * 31 + K + ra[0], alpha=1.0, lora_scale=1.25, bias=True,
+                     a_sf_range=ra, b_sf_range=rb)
+    h = host_arrays(p)
+    base = O.base_product(h["a"], h["b"], h["a_sf"], h["b_sf"], M, N, K)
+    alpha = float(2.0 ** -np.round(np.log2(np.sqrt(np.mean(base ** 2)))))
+    x = Dev(p)
+    x.alpha.fill_(alpha)
+    off = run_off(x)
+    raw = run_raw(x, x.lora_scale)
+    adp = prepare(x)
+    prep = run_prepared(x, adp)
+    finish()
+    ratio, bf = O.fold(h["lb"], p.lora_scale, alpha)
+    what = f"{kernel} {name}"
+    check_close(off, O.mm_off(h["a"], h["b"], h["a_sf"], h["b_sf"], alpha, h["bias"], M, N, K, base=base),
+                what=what + " off")
+    check_close(raw, O.mm_raw(h["a"], h["b"], h["a_sf"], h["b_sf"], alpha, h["d"], h["lb"], p.lora_scale,
+                              h["bias"], M, N, K, r, base=base), what=what + " raw")
+    check_close(prep, O.mm_prepared(h["a"], h["b"], h["a_sf"], h["b_sf"], alpha, h["d"], bf, ratio, h["bias"],
+                                    M, N, K, r, base=base), what=what + " prepared")
+
+
 def test_lora_isolation_alpha_zero():
     """alpha = 0 (the LoRA-only raw call) leaves bf16(s * d @ lora_b^T + bias)."""
     p = make_problem(200, 300, 512, 40, seed=5, alpha=0.0, lora_scale=3.0, bias=True)
@@ -349,11 +392,10 @@ def test_cfg3_sampled_prepared_and_raw():
     cols = np.unique(np.concatenate([rng.choice(p.N, 512, replace=False), np.arange(128),
                                      np.arange(p.N - 128, p.N)]))
     base = O.base_product_rows_cols(h["a"], h["b"], h["a_sf"], h["b_sf"], p.K, rows, cols)
-    d = O.bf16_bits_to_f64(h["d"].reshape(p.M, p.r))[rows]
-    lbf = O.bf16_bits_to_f64(bf.reshape(p.N, p.r))[cols]
-    lb = O.bf16_bits_to_f64(h["lb"].reshape(p.N, p.r))[cols]
-    y_prep = c["alpha"] * (base + d @ lbf.T)
-    y_raw = c["alpha"] * base + c["lora_scale"] * (d @ lb.T)
+    y_prep = O.mm_prepared(h["a"], h["b"], h["a_sf"], h["b_sf"], c["alpha"], h["d"], bf, ratio, None,
+                           p.M, p.N, p.K, p.r, base=base, rows=rows, cols=cols)
+    y_raw = O.mm_raw(h["a"], h["b"], h["a_sf"], h["b_sf"], c["alpha"], h["d"], h["lb"], c["lora_scale"], None,
+                     p.M, p.N, p.K, p.r, base=base, rows=rows, cols=cols)
     ri = torch.from_numpy(rows).cuda()
     ci = torch.from_numpy(cols).cuda()
     check_close(out[ri][:, ci], y_prep, what="cfg3 prepared")
@@ -373,7 +415,6 @@ def test_cfg4_adapter_switch_shapes(M, r):
     rows = np.arange(M) if M <= 256 else np.unique(np.concatenate([rng.choice(M, 64, replace=False), [0, M - 1]]))
     h = host_arrays(p)
     base = O.base_product_rows_cols(h["a"], h["b"], h["a_sf"], h["b_sf"], K, rows, cols)
-    d = O.bf16_bits_to_f64(h["d"].reshape(M, r))[rows]
     for lb, s in adapters:
         lbd = lb.cuda()
         sd = torch.tensor([s], dtype=torch.float32, device="cuda")
@@ -382,10 +423,11 @@ def test_cfg4_adapter_switch_shapes(M, r):
         adp = L.prepare_nvfp4_lora_adapter(lbd, sd, x.alpha)
         outp = run_prepared(x, adp, bias=False)
         finish()
-        lbf64 = O.bf16_bits_to_f64(bits(lb))[cols]
-        y = CFG4["alpha"] * base + s * (d @ lbf64.T)
+        y = O.mm_raw(h["a"], h["b"], h["a_sf"], h["b_sf"], CFG4["alpha"], h["d"], bits(lb), s, None,
+                     M, N, K, r, base=base, rows=rows, cols=cols)
         ratio, bf = O.fold(bits(lb), s, CFG4["alpha"])
-        yp = CFG4["alpha"] * (base + d @ O.bf16_bits_to_f64(bf.reshape(N, r))[cols].T)
+        yp = O.mm_prepared(h["a"], h["b"], h["a_sf"], h["b_sf"], CFG4["alpha"], h["d"], bf, ratio, None,
+                           M, N, K, r, base=base, rows=rows, cols=cols)
         ri = torch.from_numpy(rows).cuda()
         ci = torch.from_numpy(cols).cuda()
         check_close(out[ri][:, ci], y, what=f"cfg4 raw M{M} r{r}")

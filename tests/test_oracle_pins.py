@@ -374,6 +374,43 @@ def test_raw_vs_prepared_equal_when_fold_is_exact():
     np.testing.assert_allclose(y_prep, y_raw, rtol=1e-15, atol=1e-300)
 
 
+def test_sampled_call_forms_equal_the_full_forms_on_their_outputs():
+    """The rows / cols forms (used at full sizes) give exactly the selected block of the full
+    call forms, for unsorted, repeated and edge indices, with the brute-force loop as the anchor
+    of one element."""
+    p, x = _small_problem(25, M=40, N=72, K=512, r=24)
+    rows = np.array([39, 0, 17, 17, 5])
+    cols = np.array([71, 3, 0, 64, 64, 33])
+    sel = np.ix_(rows, cols)
+    s, alpha = 1.5, p.alpha
+    ratio, bf = O.fold(x["lb"], s, alpha)
+    full = {
+        "raw": O.mm_raw(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], x["lb"], s, x["bias"],
+                        p.M, p.N, p.K, p.r),
+        "prepared": O.mm_prepared(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], bf, ratio, x["bias"],
+                                  p.M, p.N, p.K, p.r),
+        "off": O.mm_off(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["bias"], p.M, p.N, p.K),
+    }
+    part = {
+        "raw": O.mm_raw(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], x["lb"], s, x["bias"],
+                        p.M, p.N, p.K, p.r, rows=rows, cols=cols),
+        "prepared": O.mm_prepared(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["d"], bf, ratio, x["bias"],
+                                  p.M, p.N, p.K, p.r, rows=rows, cols=cols),
+        "off": O.mm_off(x["a"], x["b"], x["a_sf"], x["b_sf"], alpha, x["bias"], p.M, p.N, p.K,
+                        rows=rows, cols=cols),
+    }
+    for k in full:
+        assert part[k].shape == (len(rows), len(cols)), k
+        np.testing.assert_allclose(part[k], full[k][sel], rtol=1e-14, atol=0, err_msg=k)
+    # one element of the raw form against the block-by-block sum written out here
+    m, n = 39, 71
+    a_log = O.unswizzle_scales(x["a_sf"], p.M, p.K); b_log = O.unswizzle_scales(x["b_sf"], p.N, p.K)
+    base = brute_base(x["a"][m:m + 1], x["b"][n:n + 1], a_log[m:m + 1], b_log[n:n + 1], 1, 1, p.K)[0, 0]
+    dl = p.d.double().numpy()[m] @ p.lora_b.double().numpy()[n]
+    want = alpha * base + s * dl + p.bias.double().numpy()[n]
+    assert abs(part["raw"][0, 0] - want) <= 1e-12 * max(1.0, abs(want))
+
+
 def test_measures():
     y = np.array([1.0, -2.0, 4.0])
     assert O.sqnr_db(y, y) == float("inf")

@@ -49,9 +49,12 @@ class Problem:
 def make_problem(M: int, N: int, K: int, r: int, seed: int, *, alpha: float,
                  lora_scale: Optional[float], bias: bool, d_std: float = 1.0,
                  lb_std: float = 0.02, bias_std: float = 0.1,
-                 codes: str = "uniform") -> Problem:
+                 codes: str = "uniform", a_sf_range=(SF_LO, SF_HI),
+                 b_sf_range=(SF_LO, SF_HI)) -> Problem:
     """Draw one problem.  Every byte of the padded scale buffers is drawn (padding rows
-    included), so no knowledge of the swizzle is needed here."""
+    included), so no knowledge of the swizzle is needed here.  Scale bytes are uniform over
+    the inclusive byte ranges ``a_sf_range`` / ``b_sf_range`` (default: the workloads' 0x28..0x48;
+    0x01..0x7E spans every positive finite UE4M3 value, subnormals 0x01..0x07 included)."""
     g = torch.Generator().manual_seed(seed)
     if codes == "uniform":
         a = torch.randint(0, 256, (M, K // 2), generator=g, dtype=torch.uint8)
@@ -61,8 +64,8 @@ def make_problem(M: int, N: int, K: int, r: int, seed: int, *, alpha: float,
         b = torch.zeros((N, K // 2), dtype=torch.uint8)
     else:
         raise ValueError(codes)
-    a_sf = torch.randint(SF_LO, SF_HI + 1, (sf_bytes(M, K),), generator=g, dtype=torch.uint8)
-    b_sf = torch.randint(SF_LO, SF_HI + 1, (sf_bytes(N, K),), generator=g, dtype=torch.uint8)
+    a_sf = torch.randint(a_sf_range[0], a_sf_range[1] + 1, (sf_bytes(M, K),), generator=g, dtype=torch.uint8)
+    b_sf = torch.randint(b_sf_range[0], b_sf_range[1] + 1, (sf_bytes(N, K),), generator=g, dtype=torch.uint8)
     d = (torch.randn(M, r, generator=g) * d_std).to(torch.bfloat16)
     lora_b = (torch.randn(N, r, generator=g) * lb_std).to(torch.bfloat16)
     bias_t = (torch.randn(N, generator=g) * bias_std).to(torch.bfloat16) if bias else None
