@@ -2,15 +2,17 @@
 """Throughput of the NVFP4 + LoRA GEMM on B200, against its roofline, with the CPU oracle
 timed beside it.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload cfg3] [--impl ours|reference]
 
-One step = one call of the workload's path (raw: nvfp4lora_mm; prepared: refold + GEMM for
-the adapter-switch workloads).  The default workload is the decode shape M=16, N=4096,
-K=4096, r=64 (raw path with bias), whose metric is HBM GB/s; compute-bound workloads report
-TFLOPS.  Weights are rotated through enough copies (>= 3x the L2 size in total) that every
-step reads them from HBM; steps are CUDA-graph replays timed with CUDA events on the
-launching stream.  N > 1 (torchrun): every rank runs its own independent problem (weak
-scaling, no collective on the data path); the time is the max over ranks.
+One step = one pass of the workload's path over one batch: on the prepared path the in-place
+refold of the adapter and the GEMM (two kernels), on the raw path one GEMM call.  The default
+workload is cfg3, the large MLP-up shape M=8192, N=28672, K=8192, r=64 on the prepared path,
+reported in TFLOPS against the dense FP4 peak; the same run then times the decode shape cfg1
+(M=16, N=4096, K=4096, r=64, raw path + bias), reported in HBM GB/s, as a secondary block of the
+same JSON line.  Inputs are rotated through enough copies (>= 3x the L2 size in total) that
+every step reads them from HBM; steps are CUDA-graph replays timed with CUDA events on the
+launching stream.  N > 1 (torchrun): every rank runs its own independent problem (weak scaling,
+no collective on the data path); the time is the max over ranks.
 """
 
 from __future__ import annotations
@@ -46,6 +48,9 @@ WORKLOADS = {
 
 QUANT_ROWS, QUANT_K = 8192, 8192         # cfg3's a: M x K
 
+# the workload timed after the headline one in the same run (its own block in the line)
+SECONDARY = {"cfg3": "cfg1"}
+
 
 def describe(name):
     from workloads import CFG4, CONFIGS
@@ -79,6 +84,16 @@ def upload_graph(g, stream) -> bool:
     return fn(ctypes.c_void_p(handle), ctypes.c_void_p(stream.cuda_stream)) == 0
 
 
+def hold_device(stream, us=1000.0):
+    """Enqueue a short spin on `stream` (PyTorch's own sleep kernel, outside any timed region) so
+    that the start event recorded after it is timestamped only once the host has finished
+    submitting the graph that follows: the timed region then holds the graph's kernels alone, not
+    the host's launch latency (about 20 us for a 20-call graph, a quarter of a 20-call cfg1
+    region).  Clock rate ~2 GHz; the spin length needs no precision."""
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(us * 2000))
+
+
 def time_graph(step, n, stream, device, warm=3):
     """Capture n back-to-back calls of step(i) in one CUDA graph and time one replay with CUDA
     events on the launching stream (after an untimed warm-up replay).  Returns ms per call."""
@@ -107,6 +122,7 @@ def time_graphs(steps, n, stream, device, warm=3, rounds=3):
         for name, g in graphs.items():
             start = torch.cuda.Event(enable_timing=True)
             end = torch.cuda.Event(enable_timing=True)
+            hold_device(stream)
             with torch.cuda.stream(stream):
                 start.record(stream)
                 g.replay()
@@ -243,11 +259,14 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------------------
 
-def run_ours(args, rank, world, device):
+def run_ours(args, workload, rank, world, device):
+    """Time `workload` (cfg0..cfg3): K steps in one CUDA graph on the device, then (outside the
+    timed region) the LoRA overhead against adapter-off and, on the prepared path, the raw path of
+    the same inputs, then the end-to-end run through the public API with host buffers."""
     import nvfp4_block_scaled_mm_b200 as L
     from workloads import make_problem
 
-    c = describe(args.workload)
+    c = describe(workload)
     M, N, K, r = c["M"], c["N"], c["K"], c["r"]
     p = make_problem(M, N, K, r, c["seed"] + 1000 * rank, alpha=c["alpha"], lora_scale=c["lora_scale"],
                      bias=c["bias"])
@@ -284,7 +303,7 @@ def run_ours(args, rank, world, device):
             L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, st["d"], st["lora_b"], s,
                             bias=st["bias"], out=out)
 
-    K_steps = args.steps if args.steps is not None else WORKLOADS[args.workload]["steps"]
+    K_steps = args.steps if args.steps is not None else WORKLOADS[workload]["steps"]
     W = args.warmup
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
@@ -311,6 +330,7 @@ def run_ours(args, rank, world, device):
     end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(device)
     with ClockSampler(device.index if device.index is not None else 0) as clk:
+        hold_device(stream)
         with torch.cuda.stream(stream):
             start.record(stream)
             g.replay()
@@ -323,11 +343,13 @@ def run_ours(args, rank, world, device):
     if world > 1:
         ms = max_over_ranks(ms, device)
     ms_step = ms / K_steps
+    del g, g_warm
 
     # LoRA overhead (outside the timed region): the step, the same calls without an adapter, and
-    # on the prepared path the GEMM alone with the adapter already folded, timed in turn so that
-    # clock drift falls on all of them alike
-    n_extra = min(K_steps, 2000)
+    # on the prepared path the GEMM alone with the adapter already folded and the raw path of the
+    # same inputs, timed in turn so that clock drift falls on all of them alike.  At least ~20 ms
+    # of work per graph, so that short steps are not dominated by the graph's edges.
+    n_extra = max(K_steps, min(2000, int(math.ceil(0.02 / max(ms_step * 1e-3, 1e-7)))))
 
     def step_off(i):
         st = sets[i % copies]
@@ -339,7 +361,13 @@ def run_ours(args, rank, world, device):
             st = sets[i % copies]
             L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, st["d"],
                             lora_adapter=adapters[i % copies], bias=st["bias"], out=out)
+
+        def step_raw(i):
+            st = sets[i % copies]
+            L.mm_nvfp4_lora(st["a"], st["b"], st["a_sf"], st["b_sf"], alpha, st["d"], st["lora_b"], s,
+                            bias=st["bias"], out=out)
         kinds["gemm"] = step_gemm
+        kinds["raw"] = step_raw
     t = time_graphs(kinds, n_extra, stream, device)
     overhead = {"off_ms_per_call": t["off"], "path_ms_per_step": t["path"],
                 "path_vs_off": t["path"] / t["off"] - 1.0,
@@ -347,16 +375,75 @@ def run_ours(args, rank, world, device):
     if prepared:
         overhead["gemm_ms_per_call"] = t["gemm"]
         overhead["gemm_vs_off"] = t["gemm"] / t["off"] - 1.0
+        overhead["raw_ms_per_call"] = t["raw"]
+        overhead["raw_vs_off"] = t["raw"] / t["off"] - 1.0
     L.nvfp4lora_device_status(stream)
 
     # end to end through the public API with host buffers: per step, the activation-side
     # inputs (a, a_sf, d) go host -> device and the output comes back device -> host.
     e2e = run_e2e(L, p, sets, alpha, s, out, c, device, stream, min(K_steps, 2000), prepared,
                   adapters if prepared else None)
+    if world > 1:
+        e2e["ms_step"] = max_over_ranks(e2e["ms_step"], device)
 
-    return dict(c=c, ms=ms, ms_step=ms_step, K=K_steps, W=max(W, 3), nbytes=nbytes, flops=flops, uploaded=uploaded,
-                lora_flops=lora_flops, copies=copies, clocks=clk.summary(), e2e=e2e,
-                launches=K_steps * launches_per_step, in_bytes=in_bytes, l2=l2, p=p, overhead=overhead)
+    return dict(c=c, workload=workload, ms=ms, ms_step=ms_step, K=K_steps, W=max(W, 3), nbytes=nbytes,
+                flops=flops, uploaded=uploaded, lora_flops=lora_flops, copies=copies, clocks=clk.summary(),
+                e2e=e2e, launches=K_steps * launches_per_step, in_bytes=in_bytes, l2=l2, p=p,
+                overhead=overhead)
+
+
+def roofline_block(c, workload, value, unit, nbytes, ms_total):
+    """The roofline of the workload's dominant kernel.  HBM-bound workloads: the measured copy
+    bandwidth.  Tensor-bound ones: the dense FP4 peak derived from the measured cuBLAS bf16 GEMM
+    (x 4, the nominal FP4 / bf16 ratio of 9 / 2.25 PFLOP/s), its burst figure for a timed region
+    under two seconds and its sustained figure for a longer one."""
+    peaks, peak_src = measured_peaks()
+    if unit == "GB/s":
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
+                "peak_source": f"hbm_gbs of {peak_src}"}
+    else:
+        sustained = ms_total >= 2000.0 and "bf16_tflops_sustained" in peaks
+        bf16 = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        peak = bf16 * 4.0
+        which = "bf16_tflops_sustained" if sustained else "bf16_tflops (burst; timed region %.0f ms)" % ms_total
+        roof = {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
+                "peak_source": f"{which} x 4 (nominal fp4/bf16) of {peak_src}"}
+    roof["traffic"] = recorded_traffic(workload)
+    roof["algorithmic_bytes_per_launch"] = nbytes
+    return roof
+
+
+def workload_line(args, res, world):
+    """The JSON fields of one measured workload (the headline line, or a secondary block)."""
+    c = res["c"]
+    value, unit = metric_value(c, res["nbytes"], res["flops"], res["ms_step"])
+    e2e = res["e2e"]
+    e2e_val, e2e_unit = metric_value(c, res["nbytes"], res["flops"], e2e["ms_step"])
+    line = {
+        "value": whole_job(value, world), "unit": unit, "steps": res["K"], "warmup": res["W"],
+        "ms_per_step": res["ms_step"],
+        "config": config_block(args, c, res["workload"]),
+        "roofline": roofline_block(c, res["workload"], value, unit, res["nbytes"], res["ms"]),
+        "clocks": res["clocks"],
+        "e2e": {"value": whole_job(e2e_val, world), "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms_step"], "steps": e2e["steps"],
+                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; "
+                        "step slots (4, or 2 for outputs over 64 MB) pipelined over three streams; the steps "
+                        "captured in one CUDA graph; weights resident in HBM, rotating through the same copies "
+                        "as the device-timed loop"},
+        "gpu_launches": res["launches"],
+        "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
+        "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],
+        "lora_overhead": res["overhead"],
+    }
+    ov = res["overhead"]
+    if "raw_ms_per_call" in ov:
+        # the raw path of the same inputs (the workload names it for comparison)
+        rv, ru = metric_value(c, res["nbytes"], res["flops"], ov["raw_ms_per_call"])
+        line["raw_path"] = {"value": rv, "unit": ru, "ms_per_call": ov["raw_ms_per_call"],
+                            "frac": rv / line["roofline"]["peak"], "vs_off": ov["raw_vs_off"]}
+    return line
 
 
 def cfg4_point(L, M, r, device, stream, l2, e2e=False):
@@ -750,28 +837,33 @@ def run_e2e(L, p, sets, alpha, s, out, c, device, stream, steps, prepared, adps,
 # the oracle as the CPU baseline / reference arm
 # ---------------------------------------------------------------------------------------
 
+def sample_rows(c):
+    """Output rows of the oracle's bounded sample: all of them up to 256, else the first 256 (the
+    oracle dequantises every sampled row of a on each call, so rows bound its fixed cost)."""
+    return min(c["M"], 256)
+
+
 def oracle_sample(p, c, ncols):
-    """Oracle on all M rows x the first `ncols` output columns of the workload; returns the
-    fraction of the workload's outputs this covers."""
+    """Oracle on the first `sample_rows(c)` rows x the first `ncols` output columns of the workload
+    (the oracle's own call forms, restricted to those outputs); returns the fraction of the
+    workload's outputs this covers."""
     import oracle as O
     a = p.a.numpy(); b = p.b.numpy(); a_sf = p.a_sf.numpy(); b_sf = p.b_sf.numpy()
     dbits = p.d.view(torch.int16).numpy().view(np.uint16)
     lbits = p.lora_b.view(torch.int16).numpy().view(np.uint16)
-    rows = np.arange(c["M"])
+    bias = None if p.bias is None else p.bias.view(torch.int16).numpy().view(np.uint16)
+    M, N, K, r = c["M"], c["N"], c["K"], c["r"]
+    nrows = sample_rows(c)
+    rows = np.arange(nrows)
     cols = np.arange(ncols)
-    base = O.base_product_rows_cols(a, b, a_sf, b_sf, c["K"], rows, cols)
-    dd = O.bf16_bits_to_f64(dbits.reshape(c["M"], c["r"]))
     if c["path"] == "prepared":
-        ratio, bf = O.fold(lbits[:ncols], c["lora_scale"], c["alpha"])
-        lb = O.bf16_bits_to_f64(bf.reshape(ncols, c["r"]))
-        y = c["alpha"] * (base + dd @ lb.T)
+        ratio, bf = O.fold(lbits, c["lora_scale"], c["alpha"])
+        y = O.mm_prepared(a, b, a_sf, b_sf, c["alpha"], dbits, bf, ratio, bias, M, N, K, r, rows=rows, cols=cols)
     else:
-        lb = O.bf16_bits_to_f64(lbits.reshape(c["N"], c["r"])[:ncols])
-        y = c["alpha"] * base + c["lora_scale"] * (dd @ lb.T)
-        if p.bias is not None:
-            y = y + O.bf16_bits_to_f64(p.bias.view(torch.int16).numpy().view(np.uint16)[:ncols])[None, :]
+        y = O.mm_raw(a, b, a_sf, b_sf, c["alpha"], dbits, lbits, c["lora_scale"], bias, M, N, K, r,
+                     rows=rows, cols=cols)
     O.round_output(y)
-    return ncols / c["N"]
+    return nrows * ncols / (M * N)
 
 
 def oracle_threads():
@@ -808,8 +900,8 @@ def cpu_baseline(p, c, nbytes, flops, budget_s=12.0):
     dt = time.perf_counter() - t0
     value, unit = metric_value(c, nbytes * frac / reps, flops * frac / reps, dt / reps * 1e3)
     return dict(value=value, unit=unit, cores=oracle_threads(), kind="oracle",
-                sample=f"{reps} x oracle on all {c['M']} rows x the first {ncols} of {c['N']} output columns "
-                       f"({frac / reps:.4f} of the workload each), {dt:.1f} s")
+                sample=f"{reps} x oracle on the first {sample_rows(c)} of {c['M']} rows x the first {ncols} of "
+                       f"{c['N']} output columns ({frac / reps:.5f} of the workload each), {dt:.1f} s")
 
 
 def metric_value(c, nbytes, flops, ms):
@@ -849,8 +941,9 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(args, c),
         "cpu_baseline": {"value": value, "unit": unit, "cores": oracle_threads(), "kind": "oracle",
-                         "sample": f"each step: oracle on all {c['M']} rows x the first {ncols} of {c['N']} "
-                                   f"output columns ({ncols / c['N']:.4f} of the workload)"},
+                         "sample": f"each step: oracle on the first {sample_rows(c)} of {c['M']} rows x the first "
+                                   f"{ncols} of {c['N']} output columns "
+                                   f"({sample_rows(c) * ncols / (c['M'] * c['N']):.5f} of the workload)"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -889,9 +982,11 @@ def run_reference_quant(args):
     return 0
 
 
-def config_block(args, c):
-    return {"workload": f"{args.workload}: M={c['M']} N={c['N']} K={c['K']} r={c['r']} {c['path']} path"
-                        f"{' + bias' if c['bias'] else ''}",
+def config_block(args, c, workload=None):
+    workload = workload or args.workload
+    what = "fold + GEMM per step" if c["path"] == "prepared" else "one call per step"
+    return {"workload": f"{workload}: M={c['M']} N={c['N']} K={c['K']} r={c['r']} {c['path']} path"
+                        f"{' + bias' if c['bias'] else ''} ({what})",
             "M": c["M"], "N": c["N"], "K": c["K"], "r": c["r"], "path": c["path"],
             "alpha": c["alpha"], "lora_scale": c["lora_scale"], "bias": c["bias"],
             "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU",
@@ -908,8 +1003,9 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg1")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg3")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the secondary workload's block")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -930,39 +1026,24 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return rc
-    res = run_ours(args, rank, world, device)
-    c = res["c"]
-    value, unit = metric_value(c, res["nbytes"], res["flops"], res["ms_step"])
-    peaks, peak_src = measured_peaks()
-    if unit == "GB/s":
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
-                "peak_source": f"hbm_gbs of {peak_src}"}
-    else:
-        # FP4 dense peak = measured bf16 (sustained, long step) x nominal fp4/bf16 ratio (9 / 2.25)
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 4.0
-        roof = {"bound": "tensor", "achieved": value, "peak": peak, "unit": "TFLOP/s", "frac": value / peak,
-                "peak_source": f"bf16_tflops_sustained x 4 (nominal fp4/bf16) of {peak_src}"}
-    traffic = recorded_traffic(args.workload)
-    roof["traffic"] = traffic
-    roof["algorithmic_bytes_per_launch"] = res["nbytes"]
-    e2e = res["e2e"]
-    e2e_val, e2e_unit = metric_value(c, res["nbytes"], res["flops"], e2e["ms_step"] * 1.0)
-    line = {
-        "metric": METRIC, "value": whole_job(value, world), "unit": unit, "n_gpus": world, "steps": res["K"],
-        "warmup": res["W"], "ms_per_step": res["ms_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3 -> fp32) + bf16 LoRA", "data": "synthetic",
-        "config": config_block(args, c), "roofline": roof, "clocks": res["clocks"],
-        "e2e": {"value": whole_job(e2e_val, world), "unit": e2e_unit, "h2d_bytes_per_step": e2e["h2d"],
-                "d2h_bytes_per_step": e2e["d2h"],
-                "note": "per step: a, a_sf, d host->device (pinned, one staging buffer), call, out device->host; step slots (4, or 2 for outputs over 64 MB) pipelined over three streams; the steps captured in one CUDA graph; weights resident in HBM, rotating through the same copies as the device-timed loop"},
-        "gpu_launches": res["launches"],
-        "lora_flops_per_step": res["lora_flops"], "tflops": res["flops"] / (res["ms_step"] * 1e-3) / 1e12,
-        "gbs": res["nbytes"] / (res["ms_step"] * 1e-3) / 1e9, "weight_copies": res["copies"],
-        "lora_overhead": res["overhead"],
-    }
+    # the headline workload, then (default run only) the decode workload in the same process, so
+    # that one driver run measures both regimes of the metric: TFLOPS / % of FP4 peak at large M
+    # and HBM GB/s at M <= 16
+    res = run_ours(args, args.workload, rank, world, device)
+    head = workload_line(args, res, world)
+    line = {"metric": METRIC, "value": head.pop("value"), "unit": head.pop("unit"), "n_gpus": world,
+            "steps": head.pop("steps"), "warmup": head.pop("warmup"), "ms_per_step": head.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4 (e2m1 x ue4m3 -> fp32) + bf16 LoRA", "data": "synthetic"}
+    line.update(head)
+    secondary = SECONDARY.get(args.workload) if not args.no_secondary else None
+    if secondary:
+        torch.cuda.empty_cache()
+        sec = run_ours(args, secondary, rank, world, device)
+        line["secondary"] = {secondary: workload_line(args, sec, world)}
+        line["gpu_launches"] += sec["launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(res["p"], c, res["nbytes"], res["flops"])
+        line["cpu_baseline"] = cpu_baseline(res["p"], res["c"], res["nbytes"], res["flops"])
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

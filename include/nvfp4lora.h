@@ -42,7 +42,7 @@ typedef struct CUstream_st* nvfp4lora_stream;
 typedef enum nvfp4lora_status {
     NVFP4LORA_OK = 0,
     /* Shape, pointer, alignment or size rule violated (mm_nvfp4_lora, Notes: Shape
-     * rules -- "Violations raise ValueError naming the violated requirement"). */
+     * rules): the Python layer turns it into ValueError, and the message names the rule. */
     NVFP4LORA_ERR_INVALID_ARG = 1,
     /* Prepared adapter used with another alpha, or its lora_b / lora_scale moved or
      * were written since the last (re)fold (mm_nvfp4_lora, Parameters: lora_adapter;
@@ -167,6 +167,10 @@ NVFP4LORA_API nvfp4lora_status nvfp4lora_mm_prepared(
  * Synchronises `stream`, then reads and clears the current device's error word that
  * kernels set when one of their bounded waits runs out.  Returns NVFP4LORA_OK or
  * NVFP4LORA_ERR_DEVICE_TIMEOUT (or NVFP4LORA_ERR_CUDA).
+ * The GEMM, fold and quantize calls return NVFP4LORA_OK once their work is enqueued; a kernel
+ * whose bounded wait gives up returns early and leaves its outputs (out, b_folded, ratio, codes,
+ * scales) partly unwritten.  Their contents are therefore defined only once a later
+ * nvfp4lora_device_status on the same stream has returned NVFP4LORA_OK.
  */
 NVFP4LORA_API nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream);
 
@@ -183,14 +187,15 @@ NVFP4LORA_API nvfp4lora_status nvfp4lora_selftest_wait_timeout(int64_t limit_ns,
 
 /*
  * NVFP4 quantizer: the producer of a / a_sf that the mm_nvfp4_lora page names (the paragraph
- * after the formula: "... in the 128x4 swizzled layout produced by fp4_quantize()"; Parameters:
- * alpha = alpha_base / (a_global_scale * b_global_scale)).  The pages give no rule; this library
+ * after the formula: the operands come in the 128x4 swizzled layout that fp4_quantize writes;
+ * Parameters: alpha = alpha_base / (a_global_scale * b_global_scale)).  The pages give no rule; this library
  * computes, per 16-element block along K, in float32:
  *     amax = max |x|;  sf = E4M3(rne, saturating at 448)((amax * gs) / 6);
  *     code = E2M1(rne, saturating at 6)(x * (gs / value(sf)))   (sf == 0: +0 codes),
  * so value(code) * value(sf) / gs approximates x.
  *   x       bf16 [rows, K] device, row-major, 16-byte aligned.  Finite values.
- *   global_scale  fp32 [1] device: gs, positive and finite (read on the device; no host read).
+ *   global_scale  fp32 [1] device, 4-byte aligned: gs, positive and finite (read on the device;
+ *           no host read).
  *   codes   uint8 [rows, K/2] device, caller-owned, 16-byte aligned: element 2j of a row in the
  *           low nibble of byte j.
  *   scales  uint8 device, caller-owned, 16-byte aligned, scales_bytes >= ceil(rows/128)*128*(K/16):

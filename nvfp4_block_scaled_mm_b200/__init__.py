@@ -203,6 +203,17 @@ def _need(t, name, dtype, ndim=None):
         raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
 
 
+def _same_device(anchor_name: str, anchor: torch.Tensor, **others) -> None:
+    """Every tensor given must live on the anchor tensor's device: the kernels run on that device
+    and read every operand by address there, so an operand on another GPU would be read through
+    a foreign address.  ValueError names the first tensor that differs (None entries are
+    skipped)."""
+    for name, t in others.items():
+        if t is not None and t.device != anchor.device:
+            raise ValueError(f"{name} is on {t.device} but {anchor_name} is on {anchor.device}: "
+                             "every tensor of a call must be on the same device")
+
+
 class PreparedNvFp4LoraAdapter:
     """A folded adapter (prepare_nvfp4_lora_adapter, Returns): ``b_folded`` bf16 [N, r], the
     device ``ratio`` scalar, the alpha tensor it belongs to, and the pins of its sources."""
@@ -243,6 +254,8 @@ def prepare_nvfp4_lora_adapter(lora_b: torch.Tensor, lora_scale: torch.Tensor, a
     no host read, graph-capturable; alpha must be the adapter's own alpha tensor.
     """
     _check_fold_inputs(lora_b, lora_scale, alpha)
+    _same_device("lora_b", lora_b, lora_scale=lora_scale, alpha=alpha,
+                 b_folded=None if out is None else out.b_folded, ratio=None if out is None else out.ratio)
     N, r = lora_b.shape
     stream = torch.cuda.current_stream(lora_b.device)
     if out is None:
@@ -272,6 +285,11 @@ def mm_nvfp4_lora(a: torch.Tensor, b: torch.Tensor, a_sf: torch.Tensor, b_sf: to
 
     Raw path: ``d``, ``lora_b``, ``lora_scale``; ``lora_scale=None`` is the adapter-off
     call even if d / lora_b are given.  Prepared path: ``lora_adapter=`` plus ``d``.
+
+    The call returns once the kernel is enqueued.  A kernel whose bounded wait gives up (a
+    stalled pipeline) returns early and leaves ``out`` partly unwritten, so ``out`` is defined
+    only once a later :func:`nvfp4lora_device_status` on the stream has returned without
+    raising ``DeviceTimeoutError``.
     """
     if out_dtype != torch.bfloat16:
         raise ValueError("out_dtype: only torch.bfloat16 is supported")
@@ -294,6 +312,10 @@ def mm_nvfp4_lora(a: torch.Tensor, b: torch.Tensor, a_sf: torch.Tensor, b_sf: to
         _need(bias, "bias", torch.bfloat16, 1)
         if bias.shape[0] != N:
             raise ValueError(f"bias must be [N] = [{N}]")
+    _same_device("a", a, b=b, a_sf=a_sf, b_sf=b_sf, alpha=alpha, d=d, lora_b=lora_b, lora_scale=lora_scale,
+                 bias=bias, out=out,
+                 b_folded=None if lora_adapter is None else lora_adapter.b_folded,
+                 ratio=None if lora_adapter is None else lora_adapter.ratio)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     else:
@@ -341,6 +363,7 @@ def fp4_quantize(x: torch.Tensor, global_scale: torch.Tensor, *, codes: Optional
     _need(global_scale, "global_scale", torch.float32)
     if global_scale.numel() != 1:
         raise ValueError("global_scale must be a one-element fp32 tensor")
+    _same_device("x", x, global_scale=global_scale, codes=codes, scales=scales)
     rows, K = x.shape
     if K % 64 != 0:
         raise ValueError(f"K = {K}: a multiple of 64 is required")

@@ -735,6 +735,7 @@ nvfp4lora_status nvfp4lora_quantize(const uint16_t* x, int64_t rows, int64_t K, 
                     (long long)need, (long long)scales_bytes);
     if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16))
         return fail(NVFP4LORA_ERR_INVALID_ARG, "x, codes and scales must be 16-byte aligned");
+    if (!aligned(global_scale, 4)) return fail(NVFP4LORA_ERR_INVALID_ARG, "global_scale must be 4-byte aligned");
     int dev = 0;
     DeviceInfo* info = nullptr;
     nvfp4lora_status st = device_info(&dev, &info);

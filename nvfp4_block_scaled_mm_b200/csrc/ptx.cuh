@@ -1,5 +1,5 @@
 // Inline-PTX wrappers for sm_100a: mbarriers with bounded waits, TMA / bulk copies,
-// and the tcgen05 family (TMEM alloc, scale copy, MMA, commit, load).  Written from
+// and the tcgen05 family (TMEM alloc, MMA, commit, load and store).  Written from
 // the public PTX ISA descriptions of these instructions.
 #pragma once
 
@@ -65,19 +65,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Non-blocking probe: has the phase of `parity` completed?
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-
 // Waits for the phase of `parity` to complete.  Gives up when `*abort` (if given) becomes
 // non-zero, or after `limit_ns` (default kWaitLimitNs); in the latter case it raises `*abort`
 // and the device error word.  Returns false when it gave up.
@@ -124,7 +111,7 @@ __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
 }
 
 // ------------------------------------------------------------------------------------
-// tcgen05: tensor memory, scale copy, MMA, commit, load
+// tcgen05: tensor memory, MMA, commit, load, store
 // ------------------------------------------------------------------------------------
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -153,13 +140,6 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Copy one 512-byte scale atom (32 rows x 16 bytes) from shared memory into 4 TMEM
-// columns of all 128 lanes (the 32 rows are repeated in each 32-lane quarter).
-__device__ __forceinline__ void tc_copy_scale_atom(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
 }
 
 // D(tmem) (+)= A(smem) * B(smem)^T with E2M1 operands, UE4M3 scales per 16 K-elements
@@ -258,12 +238,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
            (2ull << 61);
 }
 
-// Descriptor of one 512-byte scale atom: no swizzle, 8-row core matrices of 16-byte
-// rows, 128 bytes apart.
-__device__ __forceinline__ uint64_t sdesc_scale_atom(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFF) | (8ull << 32) | (1ull << 46);
-}
-
 // Instruction descriptor: kind::mxf4nvf4, E2M1 x E2M1, UE4M3 scales, K-major A and B,
 // M = 128, N = n.
 // Instruction descriptors with an explicit M (256 for an SM-pair MMA, cta_group::2).
@@ -290,7 +264,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int n) {
 namespace nvfp4lora {
 
 // ------------------------------------------------------------------------------------
-// thread-block clusters: rank, distributed shared memory, remote mbarrier arrival
+// thread-block clusters: rank, distributed shared-memory addresses, remote mbarrier arrival
 // ------------------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -304,20 +278,6 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
     uint32_t out;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
     return out;
-}
-
-// Callers issue a run of these loads before using any result, so that their latencies
-// overlap (each load's address comes from mapa, issued after the acquiring wait).
-__device__ __forceinline__ float ld_cluster_f32(uint32_t caddr) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr));
-    return v;
-}
-
-// Arrive on an mbarrier of another CTA of the cluster, releasing this thread's prior
-// shared-memory writes (and reads) at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
 
 // Arrival without release ordering.  Used where the arriving warp has already waited for what the
@@ -491,11 +451,6 @@ __device__ __forceinline__ void tmem_relinquish_pair() {
 
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Scale atom copy into both CTAs' TMEM, each from its own shared memory (same offsets).
-__device__ __forceinline__ void tc_copy_scale_atom_pair(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,

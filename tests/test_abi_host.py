@@ -132,6 +132,18 @@ def test_quantize_rules_are_checked_before_cuda(lib):
 
     for bad, word in ((dict(K=96), b"K"), (dict(K=0), b"K"), (dict(rows=0), b"rows"),
                       (dict(nbytes=256 * 16 - 1), b"scales needs"), (dict(x=0x10008), b"aligned"),
-                      (dict(scales=None), b"non-null"), (dict(gs=None), b"non-null")):
+                      (dict(scales=None), b"non-null"), (dict(gs=None), b"non-null"),
+                      (dict(gs=0x20002), b"global_scale must be 4-byte aligned")):
         assert call(**bad) == 1, bad
         assert word in lib.nvfp4lora_last_error(), (bad, lib.nvfp4lora_last_error())
+
+
+def test_binding_refuses_tensors_on_another_device():
+    """The binding's device rule, exercised with CPU and meta tensors (no GPU needed): an operand
+    on another device than the anchor raises ValueError naming it; None operands are skipped."""
+    import torch
+    import nvfp4_block_scaled_mm_b200 as L
+    a = torch.empty(4, device="cpu")
+    L._same_device("a", a, b=torch.empty(2, device="cpu"), d=None)
+    with pytest.raises(ValueError, match="lora_b is on meta"):
+        L._same_device("a", a, b=torch.empty(2, device="cpu"), lora_b=torch.empty(2, device="meta"))
