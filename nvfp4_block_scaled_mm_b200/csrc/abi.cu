@@ -320,15 +320,15 @@ int decode_splits(int n_tiles, int k_stages, int sms, int max_s) {
     return 1;
 }
 
-template <int MT, Mode MODE>
-nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint8_t* b, const uint8_t* a_sf,
-                                  const uint8_t* b_sf, const float* alpha, const float* scale, const uint16_t* d,
-                                  const uint16_t* lb, int64_t r, const uint16_t* bias, uint16_t* out,
-                                  int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+// STAGES ring slots (all of a split's K stages in flight where they fit); MAXS - 1 peer partial
+// slots plus one for the LoRA accumulator on rank 0.
+template <int MT, int STAGES, int MAXS, Mode MODE>
+nvfp4lora_status launch_decode_plan(DeviceInfo* info, int splits, const uint8_t* a, const uint8_t* b,
+                                    const uint8_t* a_sf, const uint8_t* b_sf, const float* alpha,
+                                    const float* scale, const uint16_t* d, const uint16_t* lb, int64_t r,
+                                    const uint16_t* bias, uint16_t* out, int64_t M, int64_t N, int64_t K,
+                                    cudaStream_t stream) {
     nvfp4lora_status st;
-    // one CTA per SM; rank 0 keeps room for MAXS - 1 peers' partials
-    constexpr int STAGES = 4;
-    constexpr int MAXS = (MT == 16) ? 8 : 4;
     auto kernel = nvfp4_decode_kernel<MT, STAGES, MAXS, MODE>;
     constexpr int smem = DecodeSmem<MT, STAGES, MAXS>::DYN_BYTES;
     if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
@@ -356,7 +356,7 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
     args.r = (int)r;
     args.n_tiles = (int)((N + 127) / 128);
     const int k_stages = (int)(K / 256);
-    args.splits = decode_splits(args.n_tiles, k_stages, info->sms, MAXS);
+    args.splits = splits;
     args.stages_per_split = k_stages / args.splits;
     args.sf_atoms_k = (int)(K / 64);
     args.sf_row_blocks_b = (int)((N + 127) / 128);
@@ -386,6 +386,26 @@ nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_b3, args);
     if (e != cudaSuccess) return cuda_fail(e, "decode GEMM launch");
     return NVFP4LORA_OK;
+}
+
+// A split cluster (S > 1) streams few K stages per CTA: 4 slots hold them all at the workload
+// shapes.  Without a split (many weight row blocks) one CTA streams the whole of K, and the ring is
+// as deep as shared memory allows, since a CTA's streaming rate is its bytes in flight over the
+// memory latency (M = 1, N = 14336, K = 4096: 10.0 us per call with 4 slots, 8.6 with 8).
+template <int MT, Mode MODE>
+nvfp4lora_status launch_decode_mt(DeviceInfo* info, const uint8_t* a, const uint8_t* b, const uint8_t* a_sf,
+                                  const uint8_t* b_sf, const float* alpha, const float* scale, const uint16_t* d,
+                                  const uint16_t* lb, int64_t r, const uint16_t* bias, uint16_t* out,
+                                  int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+    constexpr int MAXS = 4;
+    constexpr int DEEP = (MT == 16) ? 8 : 6;
+    const int n_tiles = (int)((N + 127) / 128);
+    const int splits = decode_splits(n_tiles, (int)(K / 256), info->sms, MAXS);
+    if (splits > 1)
+        return launch_decode_plan<MT, 4, MAXS, MODE>(info, splits, a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias,
+                                                     out, M, N, K, stream);
+    return launch_decode_plan<MT, DEEP, 1, MODE>(info, 1, a, b, a_sf, b_sf, alpha, scale, d, lb, r, bias, out, M,
+                                                 N, K, stream);
 }
 
 template <Mode MODE>
