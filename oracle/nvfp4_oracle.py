@@ -298,6 +298,54 @@ def mm_off(a, b, a_sf, b_sf, alpha: float, bias_bits, M: int, N: int, K: int,
     return np.float64(alpha) * base + _bias_row(bias_bits, N, cols)
 
 
+# --------------------------------------------------------------------------------------
+# Grouped (expert-partitioned) form: flashinfer.grouped_mm.grouped_mm_bf16's formula
+# (out[start:end] = a[start:end] x b[e]^T for each expert e, start, end = m_indptr[e],
+# m_indptr[e+1]) applied to this operation.  Reading taken: every m_indptr[e] is a multiple of
+# 128 (each expert's token rows fill whole 128-row blocks of the 128x4 scale layout, padding rows
+# included), alpha is per expert ([E]), lora_b ([E, N, r]) and bias ([E, N]) are per expert, d
+# and lora_scale are shared.
+# --------------------------------------------------------------------------------------
+
+def check_grouped_indptr(m_indptr, rows: int) -> np.ndarray:
+    """The reading's rules: int, starts at 0, non-decreasing, multiples of 128, ends <= rows."""
+    ind = np.asarray(m_indptr, dtype=np.int64).reshape(-1)
+    if ind.size < 2 or ind[0] != 0 or np.any(np.diff(ind) < 0) or np.any(ind % 128 != 0) or ind[-1] > rows:
+        raise ValueError("m_indptr must start at 0, be non-decreasing, hold multiples of 128 and end <= rows")
+    return ind
+
+
+def grouped_mm(a, b, a_sf, b_sf, m_indptr, alpha, d_bits, lb_bits, lora_scale, bias_bits,
+               rows: int, N: int, K: int, r: int) -> np.ndarray:
+    """float64 values of the rows [0, m_indptr[E]) of the grouped call; expert e's segment is the
+    raw-path call form (``mm_raw``; lora_scale None or 0 is adapter-off) on a[s:t] and b[e].
+
+    a: [rows, K/2]; a_sf: the 128x4 layout of all rows (so a segment's scales are its 128-row
+    blocks); b: [E, N, K/2]; b_sf: [E] consecutive scale buffers of ceil(N/128)*128*K/16 bytes;
+    alpha: [E]; d: [rows, r]; lora_b: [E, N, r]; bias: [E, N] or None."""
+    ind = check_grouped_indptr(m_indptr, rows)
+    E = ind.size - 1
+    a = np.asarray(a, dtype=np.uint8).reshape(rows, K // 2)
+    a_sf = np.asarray(a_sf, dtype=np.uint8).reshape(-1)
+    b = np.asarray(b, dtype=np.uint8).reshape(E, N, K // 2)
+    sfb_bytes = sf_buffer_bytes(N, K)
+    b_sf = np.asarray(b_sf, dtype=np.uint8).reshape(-1)
+    alpha = np.asarray(alpha, dtype=np.float64).reshape(E)
+    lb = None if lb_bits is None else np.asarray(lb_bits).reshape(E, N, r)
+    d = None if d_bits is None else np.asarray(d_bits).reshape(rows, r)
+    bias = None if bias_bits is None else np.asarray(bias_bits).reshape(E, N)
+    out = np.zeros((int(ind[-1]), N), dtype=np.float64)
+    row_sf = K // SF_VEC                        # scale bytes per row (whole 128-row blocks)
+    for e in range(E):
+        s, t = int(ind[e]), int(ind[e + 1])
+        if t == s:
+            continue
+        out[s:t] = mm_raw(a[s:t], b[e], a_sf[s * row_sf:t * row_sf], b_sf[e * sfb_bytes:(e + 1) * sfb_bytes],
+                          float(alpha[e]), None if d is None else d[s:t], None if lb is None else lb[e],
+                          lora_scale, None if bias is None else bias[e], t - s, N, K, r)
+    return out
+
+
 def round_output(y: np.ndarray) -> np.ndarray:
     """The single rounding of the fp32 result to bf16, taken here from float64."""
     return f64_to_bf16_rne(y)

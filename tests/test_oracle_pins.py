@@ -411,6 +411,52 @@ def test_sampled_call_forms_equal_the_full_forms_on_their_outputs():
     assert abs(part["raw"][0, 0] - want) <= 1e-12 * max(1.0, abs(want))
 
 
+def _grouped_inputs(seg, N, K, r, seed, bias=True):
+    rng = np.random.default_rng(seed)
+    ind = np.concatenate([[0], np.cumsum(seg)]).astype(np.int64)
+    rows = int(ind[-1]) + 128                  # rows past the last segment are padding
+    E = len(seg)
+    a = rng.integers(0, 256, (rows, K // 2), dtype=np.uint8)
+    b = rng.integers(0, 256, (E, N, K // 2), dtype=np.uint8)
+    a_sf = rng.integers(0x01, 0x7F, O.sf_buffer_bytes(rows, K), dtype=np.uint8)
+    b_sf = rng.integers(0x01, 0x7F, E * O.sf_buffer_bytes(N, K), dtype=np.uint8)
+    alpha = rng.uniform(-1, 1, E)
+    d = O.f32_to_bf16_rne(rng.standard_normal((rows, r)).astype(np.float32))
+    lb = O.f32_to_bf16_rne((0.02 * rng.standard_normal((E, N, r))).astype(np.float32))
+    bias = O.f32_to_bf16_rne((0.1 * rng.standard_normal((E, N))).astype(np.float32)) if bias else None
+    return ind, rows, a, b, a_sf, b_sf, alpha, d, lb, bias
+
+
+def test_grouped_form_against_a_brute_force_loop():
+    """Tiny grouped call (an empty expert included) against a per-row, per-element loop with the
+    closed-form decoders: expert of each row from m_indptr, its own b, scales, alpha, lora_b, bias."""
+    N, K, r = 3, 64, 8
+    ind, rows, a, b, a_sf, b_sf, alpha, d, lb, bias = _grouped_inputs([128, 0, 256], N, K, r, 31)
+    s = 0.75
+    y = O.grouped_mm(a, b, a_sf, b_sf, ind, alpha, d, lb, s, bias, rows, N, K, r)
+    a_log = O.unswizzle_scales(a_sf, rows, K)
+    dd = O.bf16_bits_to_f64(d); ll = O.bf16_bits_to_f64(lb); bb = O.bf16_bits_to_f64(bias)
+    rng = np.random.default_rng(5)
+    for m in list(rng.choice(int(ind[-1]), 40, replace=False)) + [0, 127, 128, 383]:
+        e = int(np.searchsorted(ind, m, side="right") - 1)
+        b_log = O.unswizzle_scales(b_sf[e * O.sf_buffer_bytes(N, K):(e + 1) * O.sf_buffer_bytes(N, K)], N, K)
+        for n in range(N):
+            base = brute_base(a[m:m + 1], b[e, n:n + 1], a_log[m:m + 1], b_log[n:n + 1], 1, 1, K)[0, 0]
+            want = alpha[e] * base + s * float(dd[m] @ ll[e, n]) + bb[e, n]
+            assert abs(y[m, n] - want) <= 1e-12 * max(1.0, abs(want)), (m, n)
+
+
+def test_grouped_single_expert_is_the_plain_call_and_rules_are_checked():
+    N, K, r = 40, 128, 16
+    ind, rows, a, b, a_sf, b_sf, alpha, d, lb, bias = _grouped_inputs([256], N, K, r, 32, bias=False)
+    y = O.grouped_mm(a, b, a_sf, b_sf, ind, alpha, d, lb, None, None, rows, N, K, r)
+    want = O.mm_off(a[:256], b[0], a_sf[:O.sf_buffer_bytes(256, K)], b_sf, alpha[0], None, 256, N, K)
+    np.testing.assert_array_equal(y, want)
+    for bad in ([0, 100], [128, 256], [0, 256, 128], [0, rows + 128], [0]):
+        with pytest.raises(ValueError):
+            O.check_grouped_indptr(bad, rows)
+
+
 def test_measures():
     y = np.array([1.0, -2.0, 4.0])
     assert O.sqnr_db(y, y) == float("inf")
