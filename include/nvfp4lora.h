@@ -164,6 +164,41 @@ NVFP4LORA_API nvfp4lora_status nvfp4lora_mm_prepared(
     nvfp4lora_stream stream);
 
 /*
+ * Grouped (expert-partitioned) call: flashinfer.grouped_mm.grouped_mm_bf16's formula
+ * (out[start:end] = a[start:end] x b[e]^T for each expert e, start, end = m_indptr[e],
+ * m_indptr[e+1]) applied to the operation of nvfp4lora_mm, segment by segment:
+ *     out[s:t] = bf16_rne( alpha[e] * (dequant(a[s:t]) @ dequant(b[e])^T)
+ *                          + lora_scale * (d[s:t] @ lora_b[e]^T) [+ bias[e]] )
+ *   a       uint8 [rows, K/2]; a_sf its UE4M3 scales in the 128x4 layout over all rows
+ *           (a_sf_bytes >= ceil(rows/128)*128*K/16).
+ *   b       uint8 [num_experts, N, K/2]; b_sf num_experts consecutive 128x4 buffers of N rows
+ *           (b_sf_bytes >= num_experts*ceil(N/128)*128*K/16).
+ *   m_indptr int32 [num_experts + 1] device, read on the device (no host read, graph-capturable).
+ *           Reading taken (the pages define the grouped form for bf16 only): m_indptr[0] == 0, the
+ *           entries are non-decreasing multiples of 128 and m_indptr[E] <= rows, so each expert's
+ *           rows fill whole 128-row blocks of the scale layout; padding rows inside a segment are
+ *           computed like any other row, rows from m_indptr[E] on are neither read nor written.
+ *           A table that breaks these rules computes nothing and makes the next
+ *           nvfp4lora_device_status return NVFP4LORA_ERR_INVALID_ARG.
+ *   alpha   fp32 [num_experts] device (each expert's alpha_base / (a_gs * b_gs[e])).
+ *   d       bf16 [rows, r]; lora_b bf16 [num_experts, N, r]; lora_scale fp32 [1] or NULL (adapter
+ *           off; a device value of 0 does no LoRA work and gives the adapter-off output bitwise).
+ *   bias    bf16 [num_experts, N] or NULL.   out bf16 [rows, N].
+ * Rules as for nvfp4lora_mm (alignment, K % 256 == 0, r), 1 <= num_experts <= 511.  The raw
+ * combine of nvfp4lora_mm applies per segment.  Enqueued on `stream`.
+ */
+NVFP4LORA_API nvfp4lora_status nvfp4lora_grouped_mm(
+    const uint8_t* a, const uint8_t* b,
+    const uint8_t* a_sf, int64_t a_sf_bytes,
+    const uint8_t* b_sf, int64_t b_sf_bytes,
+    const int32_t* m_indptr, int64_t num_experts,
+    const float* alpha,
+    const uint16_t* d, const uint16_t* lora_b, const float* lora_scale, int64_t r,
+    const uint16_t* bias, uint16_t* out,
+    int64_t rows, int64_t N, int64_t K,
+    nvfp4lora_stream stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error word that
  * kernels set when one of their bounded waits runs out.  Returns NVFP4LORA_OK or
  * NVFP4LORA_ERR_DEVICE_TIMEOUT (or NVFP4LORA_ERR_CUDA).

@@ -31,6 +31,7 @@ __all__ = [
     "StaleAdapterError", "PreparedNvFp4LoraAdapter", "mm_nvfp4_lora", "prepare_nvfp4_lora_adapter",
     "nvfp4lora_mm", "nvfp4lora_prepare", "nvfp4lora_refold", "nvfp4lora_mm_prepared",
     "nvfp4lora_device_status", "nvfp4lora_quantize", "fp4_quantize", "library_path", "version",
+    "nvfp4lora_grouped_mm", "grouped_mm_nvfp4_lora",
 ]
 
 OK, INVALID_ARG, STALE, ALPHA_ZERO, UNSUPPORTED_ARCH, DEVICE_TIMEOUT, CUDA_ERR = range(7)
@@ -65,6 +66,8 @@ def _load():
     lib.nvfp4lora_selftest_wait_timeout.restype = ctypes.c_int
     lib.nvfp4lora_quantize.argtypes = [P, I64, I64, P, P, P, I64, P]
     lib.nvfp4lora_quantize.restype = ctypes.c_int
+    lib.nvfp4lora_grouped_mm.argtypes = [P, P, P, I64, P, I64, P, I64, P, P, P, P, I64, P, P, I64, I64, I64, P]
+    lib.nvfp4lora_grouped_mm.restype = ctypes.c_int
     lib.nvfp4lora_last_error.argtypes = []
     lib.nvfp4lora_last_error.restype = ctypes.c_char_p
     lib.nvfp4lora_version.argtypes = []
@@ -166,6 +169,15 @@ def nvfp4lora_mm_prepared(a, b, a_sf, b_sf, alpha, d, adp, cur_lora_b, cur_lora_
                                       b_sf.numel(), _ptr(alpha), _ptr(d), ctypes.byref(adp),
                                       _ptr(cur_lora_b), _ptr(cur_lora_scale), int(cur_version),
                                       _ptr(bias), _ptr(out), int(M), int(N), int(K), _stream(stream)))
+    return out
+
+
+def nvfp4lora_grouped_mm(a, b, a_sf, b_sf, m_indptr, num_experts, alpha, d, lora_b, lora_scale, r, bias, out,
+                         rows, N, K, stream=None):
+    _check(_lib.nvfp4lora_grouped_mm(_ptr(a), _ptr(b), _ptr(a_sf), a_sf.numel(), _ptr(b_sf), b_sf.numel(),
+                                     _ptr(m_indptr), int(num_experts), _ptr(alpha), _ptr(d), _ptr(lora_b),
+                                     _ptr(lora_scale), int(r), _ptr(bias), _ptr(out), int(rows), int(N), int(K),
+                                     _stream(stream)))
     return out
 
 
@@ -349,6 +361,65 @@ def mm_nvfp4_lora(a: torch.Tensor, b: torch.Tensor, a_sf: torch.Tensor, b_sf: to
             raise ValueError(f"d must be [M, r] and lora_b [N, r]; got {tuple(d.shape)}, {tuple(lora_b.shape)}")
         nvfp4lora_mm(a, b, a_sf, b_sf, alpha, d, lora_b, lora_scale, r, bias, out, M, N, K, stream)
         return out
+
+
+def grouped_mm_nvfp4_lora(a: torch.Tensor, b: torch.Tensor, a_sf: torch.Tensor, b_sf: torch.Tensor,
+                          m_indptr: torch.Tensor, alpha: torch.Tensor, d: Optional[torch.Tensor] = None,
+                          lora_b: Optional[torch.Tensor] = None, lora_scale: Optional[torch.Tensor] = None, *,
+                          bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Grouped (expert-partitioned) form, flashinfer.grouped_mm.grouped_mm_bf16's formula applied to
+    :func:`mm_nvfp4_lora`: for each expert e with rows ``s, t = m_indptr[e], m_indptr[e+1]``,
+    ``out[s:t] = alpha[e] * (dequant(a[s:t]) @ dequant(b[e])^T) + lora_scale * (d[s:t] @ lora_b[e]^T)
+    [+ bias[e]]``.
+
+    a: uint8 [rows, K/2] with a_sf over all rows; b: uint8 [E, N, K/2] with b_sf holding E
+    consecutive 128x4 buffers; m_indptr: int32 [E + 1] on the device, 0, non-decreasing multiples
+    of 128, at most rows (each expert's rows fill whole 128-row scale blocks); alpha: fp32 [E];
+    d: bf16 [rows, r]; lora_b: bf16 [E, N, r]; lora_scale: fp32 [1] or None; bias: bf16 [E, N].
+    Rows from m_indptr[E] on are left untouched.  m_indptr is checked on the device: a table that
+    breaks its rules computes nothing, and :func:`nvfp4lora_device_status` raises ValueError.
+    """
+    _need(a, "a", torch.uint8, 2)
+    _need(b, "b", torch.uint8, 3)
+    _need(a_sf, "a_sf", torch.uint8)
+    _need(b_sf, "b_sf", torch.uint8)
+    _need(m_indptr, "m_indptr", torch.int32, 1)
+    _need(alpha, "alpha", torch.float32, 1)
+    rows, K = a.shape[0], a.shape[1] * 2
+    E, N = b.shape[0], b.shape[1]
+    if b.shape[2] * 2 != K:
+        raise ValueError(f"a is [rows, K/2] = {tuple(a.shape)} but b is {tuple(b.shape)}: K differs")
+    if m_indptr.shape[0] != E + 1 or alpha.shape[0] != E:
+        raise ValueError(f"m_indptr must be [E + 1] = [{E + 1}] and alpha [E] = [{E}]")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, 2)
+        if tuple(bias.shape) != (E, N):
+            raise ValueError(f"bias must be [E, N] = [{E}, {N}]")
+    r = 0
+    if lora_scale is not None:
+        _need(lora_scale, "lora_scale", torch.float32)
+        if lora_scale.numel() != 1:
+            raise ValueError("lora_scale must be a one-element fp32 tensor")
+        if d is None or lora_b is None:
+            raise ValueError("the LoRA term needs d and lora_b with lora_scale")
+        _need(d, "d", torch.bfloat16, 2)
+        _need(lora_b, "lora_b", torch.bfloat16, 3)
+        r = d.shape[1]
+        if d.shape[0] != rows or tuple(lora_b.shape) != (E, N, r):
+            raise ValueError(f"d must be [rows, r] and lora_b [E, N, r]; got {tuple(d.shape)}, {tuple(lora_b.shape)}")
+    if out is None:
+        out = torch.empty((rows, N), dtype=torch.bfloat16, device=a.device)
+    else:
+        _need(out, "out", torch.bfloat16, 2)
+        if tuple(out.shape) != (rows, N):
+            raise ValueError(f"out must be [rows, N] = [{rows}, {N}]")
+    _same_device("a", a, b=b, a_sf=a_sf, b_sf=b_sf, m_indptr=m_indptr, alpha=alpha, d=d, lora_b=lora_b,
+                 lora_scale=lora_scale, bias=bias, out=out)
+    with torch.cuda.device(a.device):
+        nvfp4lora_grouped_mm(a, b, a_sf, b_sf, m_indptr, E, alpha, d if lora_scale is not None else None,
+                             lora_b if lora_scale is not None else None, lora_scale, r, bias, out, rows, N, K,
+                             torch.cuda.current_stream(a.device))
+    return out
 
 
 def fp4_quantize(x: torch.Tensor, global_scale: torch.Tensor, *, codes: Optional[torch.Tensor] = None,

@@ -289,6 +289,8 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     args.sf_atoms_k = (int)(K / 64);
     args.sf_row_blocks_b = (int)((N + 127) / 128);
     args.vec_out = vec_out ? 1 : 0;
+    args.m_indptr = nullptr;
+    args.num_experts = 0;
 
     const int grid = (int)std::min<int64_t>(tiles, info->sms);
     cudaLaunchConfig_t cfg = {};
@@ -303,6 +305,80 @@ nvfp4lora_status launch_gemm(const uint8_t* a, const uint8_t* b, const uint8_t* 
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_out, args);
     if (e != cudaSuccess) return cuda_fail(e, "GEMM launch");
+    return NVFP4LORA_OK;
+}
+
+// Grouped call (nvfp4lora_grouped_mm): the single-SM tiled kernel over 128-row blocks whose expert
+// comes from m_indptr on the device.  `rows` is the row count of a, d and out; b and lora_b are
+// [E * N, .] row-major; alpha is [E].
+template <Mode MODE>
+nvfp4lora_status launch_gemm_grouped(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, const uint8_t* b_sf,
+                                     const int* m_indptr, int64_t E, const float* alpha, const float* scale,
+                                     const uint16_t* d, const uint16_t* lb, int64_t r, const uint16_t* bias,
+                                     uint16_t* out, int64_t rows, int64_t N, int64_t K, cudaStream_t stream) {
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+
+    auto kernel = nvfp4_gemm_kernel<kStages, MODE, true>;
+    constexpr int smem = GemmSmem<kStages>::DYN_BYTES;
+    if ((st = ensure_smem_attr(info, kernel, smem)) != NVFP4LORA_OK) return st;
+    static std::atomic<int> regs_ok{0};            // one per instantiation
+    if ((st = check_split_regs(kernel, kGemmRegsLaunch, regs_ok, "grouped GEMM")) != NVFP4LORA_OK) return st;
+
+    CUtensorMap tm_a, tm_b, tm_d, tm_lb, tm_out;
+    std::memset(&tm_d, 0, sizeof(tm_d));
+    std::memset(&tm_lb, 0, sizeof(tm_lb));
+    std::memset(&tm_out, 0, sizeof(tm_out));
+    if ((st = encode_2d(&tm_a, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, rows, 128, kTileM)) != NVFP4LORA_OK) return st;
+    if ((st = encode_2d(&tm_b, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, E * N, 128, kTileN)) != NVFP4LORA_OK) return st;
+    if (MODE != Mode::Off) {
+        if ((st = encode_2d(&tm_d, d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, rows, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B, kLoraPromotion)) != NVFP4LORA_OK) return st;
+        if ((st = encode_2d(&tm_lb, lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, E * N, 64, kTileN, CU_TENSOR_MAP_SWIZZLE_128B, kLoraPromotion)) != NVFP4LORA_OK) return st;
+    }
+    const bool vec_out = (N % 8 == 0 && (bias == nullptr || aligned(bias, 16)));
+    if (vec_out &&
+        (st = encode_2d(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, rows, kOutBoxCols, kOutBoxRows,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NVFP4LORA_OK)
+        return st;
+
+    GemmArgs args;
+    args.a_sf = a_sf;
+    args.b_sf = b_sf;
+    args.alpha = alpha;
+    args.scale = scale;
+    args.bias = bias;
+    args.out = out;
+    args.M = (int)rows;
+    args.N = (int)N;
+    args.K = (int)K;
+    args.r = (int)r;
+    args.m_tiles = (int)((rows + kTileM - 1) / kTileM);     // bound: the kernel reads m_indptr[E]
+    args.n_tiles = (int)((N + kTileN - 1) / kTileN);
+    const int64_t tiles = (int64_t)args.m_tiles * args.n_tiles;
+    if (tiles > INT32_MAX) return fail(NVFP4LORA_ERR_INVALID_ARG, "too many output tiles (rows x N too large)");
+    args.num_tiles = (int)tiles;
+    args.k_stages = (int)(K / 256);
+    args.sf_atoms_k = (int)(K / 64);
+    args.sf_row_blocks_b = (int)((N + 127) / 128);         // per expert
+    args.vec_out = vec_out ? 1 : 0;
+    args.m_indptr = m_indptr;
+    args.num_experts = (int)E;
+
+    const int grid = (int)std::min<int64_t>(tiles, info->sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_d, tm_lb, tm_out, args);
+    if (e != cudaSuccess) return cuda_fail(e, "grouped GEMM launch");
     return NVFP4LORA_OK;
 }
 
@@ -708,6 +784,41 @@ nvfp4lora_status nvfp4lora_mm_prepared(const uint8_t* a, const uint8_t* b, const
                                        adapter->r, bias, out, M, N, K, reinterpret_cast<cudaStream_t>(stream));
 }
 
+nvfp4lora_status nvfp4lora_grouped_mm(const uint8_t* a, const uint8_t* b, const uint8_t* a_sf, int64_t a_sf_bytes,
+                                      const uint8_t* b_sf, int64_t b_sf_bytes, const int32_t* m_indptr,
+                                      int64_t num_experts, const float* alpha, const uint16_t* d,
+                                      const uint16_t* lora_b, const float* lora_scale, int64_t r,
+                                      const uint16_t* bias, uint16_t* out, int64_t rows, int64_t N, int64_t K,
+                                      nvfp4lora_stream stream) {
+    t_last_error.clear();
+    if (num_experts < 1 || num_experts > kMaxExperts)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "num_experts = %lld: 1 <= num_experts <= %d is required",
+                    (long long)num_experts, kMaxExperts);
+    if (rows > kMaxDim || (int64_t)num_experts * N > kMaxDim)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "rows and num_experts x N must be at most 2^30");
+    // the per-expert scale buffers of b are consecutive, ceil(N/128)*128*K/16 bytes each
+    const int64_t per_expert_sf = (N + 127) / 128 * 128 * (K / 16);
+    nvfp4lora_status st = check_base(a, b, a_sf, a_sf_bytes, b_sf, per_expert_sf, alpha, bias, out, rows, N, K);
+    if (st != NVFP4LORA_OK) return st;
+    if (b_sf_bytes < num_experts * per_expert_sf)
+        return fail(NVFP4LORA_ERR_INVALID_ARG,
+                    "b_sf has %lld bytes; num_experts consecutive 128x4 buffers of N rows need %lld",
+                    (long long)b_sf_bytes, (long long)(num_experts * per_expert_sf));
+    if (!m_indptr || !aligned(m_indptr, 4))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "m_indptr must be a non-null, 4-byte aligned int32 array");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (lora_scale == nullptr)
+        return launch_gemm_grouped<Mode::Off>(a, b, a_sf, b_sf, m_indptr, num_experts, alpha, nullptr, nullptr,
+                                              nullptr, 0, bias, out, rows, N, K, s);
+    if ((st = check_rank(r)) != NVFP4LORA_OK) return st;
+    if (!d || !lora_b) return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_scale given: d and lora_b must be non-null");
+    if (!aligned(d, 16) || !aligned(lora_b, 16))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "d and lora_b must be 16-byte aligned");
+    if (!aligned(lora_scale, 4)) return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_scale must be 4-byte aligned");
+    return launch_gemm_grouped<Mode::Raw>(a, b, a_sf, b_sf, m_indptr, num_experts, alpha, lora_scale, d, lora_b, r,
+                                          bias, out, rows, N, K, s);
+}
+
 nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream) {
     t_last_error.clear();
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
@@ -719,6 +830,10 @@ nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream) {
         const int zero = 0;
         e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
         if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+        if (word == kErrBadIndptr)
+            return fail(NVFP4LORA_ERR_INVALID_ARG,
+                        "grouped call: m_indptr must start at 0, be non-decreasing, hold multiples of 128 and "
+                        "end at most at the row count (no tile was computed)");
         return fail(NVFP4LORA_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (pipeline stalled)");
     }
     return NVFP4LORA_OK;

@@ -52,7 +52,26 @@ struct GemmArgs {
     int sf_atoms_k;          // K / 64: 512-byte scale atoms per 128-row block
     int sf_row_blocks_b;     // ceil(N / 128): 128-row scale blocks present in b_sf
     int vec_out;             // 1: rows of out (and bias) may be written / read 16 bytes at a time
+    // grouped call (the GROUPED instantiation only): expert e owns rows [m_indptr[e],
+    // m_indptr[e+1]) of a, d and out, rows [e*N, (e+1)*N) of b and lora_b, scale blocks
+    // [e*sf_row_blocks_b, (e+1)*sf_row_blocks_b) of b_sf, alpha[e] and bias[e*N, (e+1)*N)
+    const int* m_indptr;     // [num_experts + 1], device; multiples of 128, read on the device
+    int num_experts;
 };
+
+constexpr int kMaxExperts = 511;         // grouped call: m_indptr lives in shared memory
+constexpr int kErrBadIndptr = 2;         // device error word: a grouped call's m_indptr broke its rules
+
+// Largest e in [0, E) with ind[e] <= row, for non-decreasing ind with ind[0] <= row < ind[E]: the
+// expert whose rows hold `row` (empty experts, ind[e] == ind[e + 1], are skipped).
+__device__ __forceinline__ int expert_of_row(const int* ind, int E, int row) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (ind[mid] <= row) lo = mid; else hi = mid;
+    }
+    return lo;
+}
 
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
@@ -92,10 +111,13 @@ struct GemmSmem {
     static constexpr int OUT_OFF = BIAS_OFF + 2 * BIAS_BYTES;
     static constexpr int BAR_OFF = OUT_OFF + kEpiWarps * kOutBoxes * OUT_BOX_BYTES;
     static constexpr int MAX_SLOTS = 8;                  // TMEM scale slots (at most)
+    // grouped call: m_indptr copied from global memory, then [rows / 128 in use, valid]
+    static constexpr int IND_OFF = BAR_OFF;
+    static constexpr int IND_BYTES = (kMaxExperts + 1) * 4 + 16;
     // full[S], empty[S], sf_full[SF], sf_empty[SF], sf_ready[8], slot_free[8], tmem_full,
-    // acc_empty, lacc_full, lacc_empty, drain, bias_full[2], bias_empty[2]
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * kSfStages + 2 * MAX_SLOTS + 9;
-    static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+    // acc_empty, lacc_full, lacc_empty, drain, bias_full[2], bias_empty[2], groups_ready
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * kSfStages + 2 * MAX_SLOTS + 10;
+    static constexpr int MISC_OFF = BAR_OFF + IND_BYTES + NUM_BARS * 8;
     static constexpr int TOTAL = MISC_OFF + 16;
     static constexpr int DYN_BYTES = TOTAL + 1024;    // slack to align the base to 1024 bytes
     static_assert(DYN_BYTES <= 232448, "shared-memory plan exceeds 227 KB");
@@ -124,7 +146,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int STAGES, Mode MODE>
+template <int STAGES, Mode MODE, bool GROUPED = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   const __grid_constant__ CUtensorMap tm_d, const __grid_constant__ CUtensorMap tm_lb,
@@ -140,7 +162,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF + L::IND_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* sf_full = empty + STAGES;           // a stage's scale atoms are in shared memory
     uint64_t* sf_empty = sf_full + kSfStages;     // ... and the staging warps have read them
@@ -153,6 +175,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     uint64_t* drain = lacc_empty + 1;
     uint64_t* bias_full = drain + 1;              // [2]: a tile's bias values are in shared memory
     uint64_t* bias_empty = bias_full + 2;         // [2]: ... and every epilogue thread has read them
+    uint64_t* groups_ready = bias_empty + 2;      // grouped call: m_indptr is in shared memory
+    int* ind = reinterpret_cast<int*>(smem + L::IND_OFF);   // grouped: m_indptr, then [m_tiles, valid]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
 
@@ -185,6 +209,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             mbar_init(&bias_full[k], 1);
             mbar_init(&bias_empty[k], 32 * kEpiWarps);
         }
+        mbar_init(groups_ready, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -192,6 +217,24 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         tmem_alloc(tmem_slot, T::ALLOC);
         tmem_relinquish();
     }
+    const int E = GROUPED ? args.num_experts : 1;
+    // The tile grid: (m blocks of 128 rows) x (n blocks of 256 columns), m fastest.  A grouped call
+    // takes its rows, [0, m_indptr[E]), from the table warp 3 puts in shared memory (no tiles at all
+    // when m_indptr breaks its rules); every role reads the same values.
+    auto tile_grid = [&](int& m_tiles, int& num_tiles) -> bool {
+        if constexpr (!GROUPED) {
+            m_tiles = args.m_tiles;
+            num_tiles = args.num_tiles;
+            return true;
+        } else {
+            m_tiles = 0;
+            num_tiles = 0;
+            if (!mbar_wait(groups_ready, 0, abort_flag)) return false;
+            m_tiles = ind[kMaxExperts + 1];
+            num_tiles = m_tiles * args.n_tiles;
+            return true;
+        }
+    };
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -205,7 +248,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         reg_dealloc<kGemmRegsCtl>();
         if (warp == 0 && lane == 0) {
             // ------------------------------- TMA producer -------------------------------
-            if (blockIdx.x < args.num_tiles) {
+            if (!GROUPED && blockIdx.x < args.num_tiles) {
                 // warm L2 with the first stages of this CTA's first tile (a prefetch changes no
                 // data, so it may precede the dependency wait)
                 const int m_blk = blockIdx.x % args.m_tiles, n_blk = blockIdx.x / args.m_tiles;
@@ -223,13 +266,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             }
             int stage = 0;
             uint32_t phase = 0, filled = 0, filled_parity = 0;
-            bool ok = true;
+            int m_tiles, num_tiles;
+            bool ok = tile_grid(m_tiles, num_tiles);
             const bool bias_smem = args.bias != nullptr && args.vec_out;
             int tl = 0;                                // local tile counter
             uint32_t bias_issued = 0, bias_par = 0;    // per buffer: issued, parity of its last phase
-            for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x, ++tl) {
-                const int m_blk = tile % args.m_tiles;
-                const int n_blk = tile / args.m_tiles;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++tl) {
+                const int m_blk = tile % m_tiles;
+                const int n_blk = tile / m_tiles;
+                const int e = GROUPED ? expert_of_row(ind, E, m_blk * kTileM) : 0;
+                const int b_row = e * args.N + n_blk * kTileN;     // this tile's rows of b / lora_b
                 const int items = args.k_stages + (sv != 0.0f ? lora_chunks_if_on : 0);
                 if (bias_smem) {
                     // the tile's bias slice, once the epilogue of two tiles ago has read the buffer
@@ -238,7 +284,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     const int n0 = n_blk * kTileN;
                     const uint32_t bytes = (uint32_t)min(kTileN, args.N - n0) * 2u;   // N % 8 == 0
                     mbar_arrive_expect_tx(&bias_full[bb], bytes);
-                    bulk_load(smem + L::BIAS_OFF + bb * L::BIAS_BYTES, args.bias + n0, bytes, &bias_full[bb]);
+                    bulk_load(smem + L::BIAS_OFF + bb * L::BIAS_BYTES, args.bias + (size_t)e * args.N + n0, bytes,
+                              &bias_full[bb]);
                     bias_issued |= 1u << bb;
                     bias_par = (bias_par & ~(1u << bb)) | ((((uint32_t)tl >> 1) & 1u) << bb);
                 }
@@ -250,10 +297,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                     if (it >= args.k_stages) {
                         const int c = it - args.k_stages;
                         tma_load_2d(sa, &tm_d, &full[stage], c * 64, m_blk * kTileM);
-                        tma_load_2d(sb, &tm_lb, &full[stage], c * 64, n_blk * kTileN);
+                        tma_load_2d(sb, &tm_lb, &full[stage], c * 64, b_row);
                     } else {
                         tma_load_2d(sa, &tm_a, &full[stage], it * 128, m_blk * kTileM);
-                        tma_load_2d(sb, &tm_b, &full[stage], it * 128, n_blk * kTileN);
+                        tma_load_2d(sb, &tm_b, &full[stage], it * 128, b_row);
                     }
                     filled |= 1u << stage;
                     filled_parity = (filled_parity & ~(1u << stage)) | (phase << stage);
@@ -276,12 +323,15 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             grid_dependency_wait();
             int sst = 0;
             uint32_t sphase = 0, issued = 0, issued_par = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
-                const int m_blk = tile % args.m_tiles;
-                const int n_blk = tile / args.m_tiles;
-                const int rb0 = n_blk * (kTileN / 128);
-                const int nsfb = (rb0 + 1 < args.sf_row_blocks_b) ? 2 : 1;
+            int m_tiles, num_tiles;
+            bool ok = tile_grid(m_tiles, num_tiles);
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int m_blk = tile % m_tiles;
+                const int n_blk = tile / m_tiles;
+                const int e = GROUPED ? expert_of_row(ind, E, m_blk * kTileM) : 0;
+                const int rbl = n_blk * (kTileN / 128);     // the tile's first 128-row block of B
+                const int nsfb = (rbl + 1 < args.sf_row_blocks_b) ? 2 : 1;
+                const int rb0 = e * args.sf_row_blocks_b + rbl;
                 for (int it = 0; it < args.k_stages; ++it) {
                     if (!mbar_wait(&sf_empty[sst], sphase ^ 1, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(&sf_full[sst], 2048u + (uint32_t)nsfb * 2048u);
@@ -308,9 +358,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             if constexpr (MODE != Mode::Off) sv = *args.scale;
             int stage = 0, slot = 0;
             uint32_t phase = 0, slot_use = 0, lacc_waits = 0;
-            bool ok = true;
+            int m_tiles, num_tiles;
+            bool ok = tile_grid(m_tiles, num_tiles);
             int i = 0;   // local tile counter
-            for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x, ++i) {
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++i) {
                 if (!mbar_wait(acc_empty, (i & 1) ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 // base product: k_stages x 4 MMAs of 128 x 256 x 64
@@ -392,6 +443,27 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 tc_commit(drain);
                 mbar_wait(drain, 0, nullptr);
             }
+        } else if (GROUPED && warp == 3) {
+            // --------------------- grouped call: m_indptr into shared memory ---------------------
+            // Its rules (the grouped reading of the 128x4 layout): m_indptr[0] == 0, non-decreasing,
+            // every entry a multiple of 128 and at most M (the rows of a, d and out).  A table that
+            // breaks them gives no tiles and raises the device error word.
+            grid_dependency_wait();
+            bool valid = true;
+            for (int k = lane; k <= E; k += 32) {
+                const int v = args.m_indptr[k];
+                ind[k] = v;
+                if (v < 0 || v % kTileM != 0 || v > args.M) valid = false;
+                if (k == 0 && v != 0) valid = false;
+                if (k > 0 && v < args.m_indptr[k - 1]) valid = false;
+            }
+            valid = __all_sync(kAll, valid);
+            __syncwarp();
+            if (lane == 0) {
+                ind[kMaxExperts + 1] = valid ? ind[E] / kTileM : 0;
+                if (!valid) atomicExch(&g_device_error, kErrBadIndptr);
+                mbar_arrive(groups_ready);
+            }
         }
         __syncwarp();
     } else if (wg == 1) {
@@ -405,8 +477,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         grid_dependency_wait();
         int sst = 0;
         uint32_t sphase = 0, g = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < args.num_tiles; tile += gridDim.x) {
+        int m_tiles, num_tiles;
+        bool ok = __all_sync(kAll, tile_grid(m_tiles, num_tiles));
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
             for (int it = 0; it < args.k_stages; ++it) {
                 const uint32_t slot = g % T::NSF, use = g / T::NSF;
                 if (!__all_sync(kAll, mbar_wait(&sf_full[sst], sphase, abort_flag))) { ok = false; break; }
@@ -454,11 +527,16 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         float lora_s = 0.0f;
         if constexpr (MODE != Mode::Off) lora_s = *args.scale;
         const bool lora_on = (MODE != Mode::Off) && lora_s != 0.0f;
-        const float alpha = *args.alpha;
+        const float alpha0 = *args.alpha;
+        int m_tiles, num_tiles;
+        const bool grid_ok = __all_sync(kAll, tile_grid(m_tiles, num_tiles));
         int i = 0, out_box = 0;
-        for (int tile = blockIdx.x; tile < args.num_tiles; tile += gridDim.x, ++i) {
-            const int m_blk = tile % args.m_tiles;
-            const int n_blk = tile / args.m_tiles;
+        for (int tile = blockIdx.x; grid_ok && tile < num_tiles; tile += gridDim.x, ++i) {
+            const int m_blk = tile % m_tiles;
+            const int n_blk = tile / m_tiles;
+            const int e = GROUPED ? expert_of_row(ind, E, m_blk * kTileM) : 0;
+            const float alpha = GROUPED ? args.alpha[e] : alpha0;     // per expert in a grouped call
+            const uint16_t* bias = (args.bias != nullptr) ? args.bias + (size_t)e * args.N : nullptr;
             if (!__all_sync(kAll, mbar_wait(tmem_full, i & 1, abort_flag))) break;
             tc_fence_after();
             uint32_t raw[128];
@@ -489,7 +567,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             }
             const int row = m_blk * kTileM + rl;
             const int col0 = n_blk * kTileN + h * 128;
-            if (args.bias != nullptr) {
+            if (bias != nullptr) {
                 if (args.vec_out) {
                     // the producer put the tile's bias slice in shared memory (past N the values
                     // are stale, and those columns are clipped by the TMA store)
@@ -511,7 +589,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
 #pragma unroll
                     for (int k = 0; k < 128; ++k)
                         if (col0 + k < args.N)
-                            v[k] = __fadd_rn(v[k], __uint_as_float((uint32_t)__ldg(args.bias + col0 + k) << 16));
+                            v[k] = __fadd_rn(v[k], __uint_as_float((uint32_t)__ldg(bias + col0 + k) << 16));
                 }
             }
             if (args.vec_out) {

@@ -147,3 +147,26 @@ def test_binding_refuses_tensors_on_another_device():
     L._same_device("a", a, b=torch.empty(2, device="cpu"), d=None)
     with pytest.raises(ValueError, match="lora_b is on meta"):
         L._same_device("a", a, b=torch.empty(2, device="cpu"), lora_b=torch.empty(2, device="meta"))
+
+
+def test_grouped_rules_are_checked_before_cuda(lib):
+    f = lib.nvfp4lora_grouped_mm
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, I64, P, I64, P, I64, P, P, P, P, I64, P, P, I64, I64, I64, P]
+    lib.nvfp4lora_last_error.restype = ctypes.c_char_p
+    ok = dict(a=0x10000, b=0x20000, a_sf=0x30000, a_sf_bytes=1 << 30, b_sf=0x40000, b_sf_bytes=1 << 30,
+              ind=0x50000, E=4, alpha=0x60000, d=0x70000, lb=0x80000, s=0x90000, r=16, bias=None,
+              out=0xA0000, rows=512, N=256, K=256)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["a"], a["b"], a["a_sf"], a["a_sf_bytes"], a["b_sf"], a["b_sf_bytes"], a["ind"], a["E"],
+                 a["alpha"], a["d"], a["lb"], a["s"], a["r"], a["bias"], a["out"], a["rows"], a["N"], a["K"], None)
+
+    for bad, word in ((dict(E=0), b"num_experts"), (dict(E=512), b"num_experts"), (dict(ind=None), b"m_indptr"),
+                      (dict(ind=0x50002), b"m_indptr"), (dict(b_sf_bytes=4 * 256 * 16 - 1), b"b_sf"),
+                      (dict(K=200), b"K = 200"), (dict(r=12), b"rank"), (dict(d=None), b"non-null"),
+                      (dict(a_sf_bytes=512 * 16 - 1), b"a_sf")):
+        assert call(**bad) == 1, bad
+        assert word in lib.nvfp4lora_last_error(), (bad, lib.nvfp4lora_last_error())

@@ -72,6 +72,49 @@ def make_problem(M: int, N: int, K: int, r: int, seed: int, *, alpha: float,
     return Problem(M, N, K, r, a, b, a_sf, b_sf, alpha, lora_scale, d, lora_b, bias_t)
 
 
+@dataclasses.dataclass
+class GroupedProblem:
+    """One grouped (expert-partitioned) problem's host tensors: expert e owns rows
+    [m_indptr[e], m_indptr[e+1]) of a, d and out."""
+    rows: int
+    N: int
+    K: int
+    r: int
+    m_indptr: torch.Tensor   # int32 [E + 1]
+    a: torch.Tensor          # uint8 [rows, K/2]
+    b: torch.Tensor          # uint8 [E, N, K/2]
+    a_sf: torch.Tensor       # uint8, the padded swizzled layout of all rows, drawn bytewise
+    b_sf: torch.Tensor       # uint8, E consecutive padded buffers, drawn bytewise
+    alpha: torch.Tensor      # fp32 [E]
+    d: torch.Tensor          # bf16 [rows, r]
+    lora_b: torch.Tensor     # bf16 [E, N, r]
+    bias: Optional[torch.Tensor]   # bf16 [E, N]
+
+
+def make_grouped_problem(segments, N: int, K: int, r: int, seed: int, *, pad_rows: int = 128,
+                         bias: bool = True, sf_range=(SF_LO, SF_HI), alpha_range=(2.0 ** -10, 2.0 ** -6),
+                         lb_std: float = 0.02, bias_std: float = 0.1) -> GroupedProblem:
+    """Draw a grouped problem whose expert e has segments[e] rows (multiples of 128 by the grouped
+    reading); `pad_rows` rows past the last segment belong to no expert.  Draw order: a, b, a_sf,
+    b_sf, alpha, d, lora_b, bias."""
+    g = torch.Generator().manual_seed(seed)
+    E = len(segments)
+    offs = [0]
+    for n in segments:
+        offs.append(offs[-1] + int(n))
+    rows = offs[-1] + pad_rows
+    a = torch.randint(0, 256, (rows, K // 2), generator=g, dtype=torch.uint8)
+    b = torch.randint(0, 256, (E, N, K // 2), generator=g, dtype=torch.uint8)
+    a_sf = torch.randint(sf_range[0], sf_range[1] + 1, (sf_bytes(rows, K),), generator=g, dtype=torch.uint8)
+    b_sf = torch.randint(sf_range[0], sf_range[1] + 1, (E * sf_bytes(N, K),), generator=g, dtype=torch.uint8)
+    alpha = torch.empty(E).uniform_(alpha_range[0], alpha_range[1], generator=g).to(torch.float32)
+    d = torch.randn(rows, r, generator=g).to(torch.bfloat16)
+    lora_b = (torch.randn(E, N, r, generator=g) * lb_std).to(torch.bfloat16)
+    bias_t = (torch.randn(E, N, generator=g) * bias_std).to(torch.bfloat16) if bias else None
+    return GroupedProblem(rows, N, K, r, torch.tensor(offs, dtype=torch.int32), a, b, a_sf, b_sf, alpha, d,
+                          lora_b, bias_t)
+
+
 def make_adapters(N: int, r: int, count: int, seed: int, lb_std: float = 0.02):
     """``count`` adapters: lora_b ~ N(0, lb_std) bf16 [N, r], lora_scale ~ U[0.1, 4]."""
     g = torch.Generator().manual_seed(seed)
