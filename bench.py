@@ -44,6 +44,7 @@ WORKLOADS = {
     "cfg3": dict(src="cfg3", steps=100),
     "cfg4": dict(src=None, steps=None),   # adapter-switch sweep (its own runner)
     "quant": dict(src=None, steps=400),   # the NVFP4 quantizer on the cfg3 activations (its own runner)
+    "moe": dict(src=None, steps=200),     # the grouped call on an 8-expert layer (its own runner)
 }
 
 QUANT_ROWS, QUANT_K = 8192, 8192         # cfg3's a: M x K
@@ -167,16 +168,17 @@ def measured_peaks():
 
 
 def source_hash(kernel="gemm"):
-    """Hash of the sources a kernel's recorded ncu figures depend on: its own kernel files and the
-    host launcher (abi.cu).  The GEMM kernels depend on every source but the quantizer's."""
+    """Hash of the kernel sources a recorded ncu figure depends on: the GEMM kernels (tiled, SM-pair,
+    decode), the fold and the PTX wrappers for `gemm`, the quantizer and the wrappers for
+    `quantize`.  The host launcher is not hashed: a change of a launch configuration there is
+    re-captured by hand."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "nvfp4_block_scaled_mm_b200", "csrc")
-    files = sorted(os.listdir(d))
     if kernel == "quantize":
-        files = ["abi.cu", "quantize.cuh"]
+        files = ["ptx.cuh", "quantize.cuh"]
     else:
-        files = [f for f in files if f != "quantize.cuh"]
+        files = ["fold.cuh", "gemm.cuh", "gemm_decode.cuh", "gemm_pair.cuh", "ptx.cuh"]
     for f in files:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
@@ -566,6 +568,209 @@ def run_cfg4(args, rank, world, device):
     return 0
 
 
+def moe_algorithmic(mp):
+    """Algorithmic bytes and flops of one grouped call (rows past m_indptr[E] are not touched)."""
+    E = mp.b.shape[0]
+    used = int(mp.m_indptr[-1])
+    N, K, r = mp.N, mp.K, mp.r
+    nbytes = (used * K // 2 + E * N * K // 2 + used * K // 16 + E * N * K // 16 + used * r * 2 + E * N * r * 2
+              + (E * N * 2 if mp.bias is not None else 0) + used * N * 2 + 4 * E + 4 * (E + 1) + 4)
+    return nbytes, 2 * used * N * K
+
+
+def moe_oracle_sample(mp, ncols):
+    """The oracle's raw call form on expert 0's first 128 rows x the first `ncols` columns (the same
+    definition the grouped form applies per segment); returns the fraction of the layer's outputs."""
+    import oracle as O
+    from workloads import MOE
+    K, N, r = mp.K, mp.N, mp.r
+    rows = 128
+    sfb = O.sf_buffer_bytes(N, K)
+    O.round_output(O.mm_raw(mp.a.numpy()[:rows], mp.b.numpy()[0], mp.a_sf.numpy()[:rows * K // 16],
+                            mp.b_sf.numpy()[:sfb], float(mp.alpha[0]),
+                            mp.d.view(torch.int16).numpy().view(np.uint16)[:rows],
+                            mp.lora_b.view(torch.int16).numpy().view(np.uint16)[0], MOE["lora_scale"],
+                            None if mp.bias is None else mp.bias.view(torch.int16).numpy().view(np.uint16)[0],
+                            rows, N, K, r, cols=np.arange(ncols)))
+    return rows * ncols / (int(mp.m_indptr[-1]) * N)
+
+
+def moe_cpu_value(mp, budget_s):
+    """Oracle throughput (TFLOPS) on bounded samples for about budget_s seconds, and the sample text."""
+    _, flops = moe_algorithmic(mp)
+    ncols = 64
+    t0 = time.perf_counter()
+    moe_oracle_sample(mp, ncols)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    ncols = max(8, min(mp.N, int(ncols * budget_s / 3 / dt)))
+    t0 = time.perf_counter()
+    reps, frac = 0, 0.0
+    while True:
+        frac += moe_oracle_sample(mp, ncols)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    value = flops * frac / dt / 1e12
+    return value, (f"{reps} x oracle raw call form on expert 0's first 128 rows x the first {ncols} of {mp.N} "
+                   f"columns ({frac / reps:.5f} of the layer each), {dt:.1f} s"), dt
+
+
+def run_moe(args, rank, world, device):
+    """The grouped call on an 8-expert layer (workloads.MOE): raw path with per-expert bias, inputs
+    rotated through copies totalling >= 3x L2, K calls in one CUDA graph timed with CUDA events."""
+    import nvfp4_block_scaled_mm_b200 as L
+    from workloads import MOE, make_grouped_problem
+    mp = make_grouped_problem(list(MOE["segments"]), MOE["N"], MOE["K"], MOE["r"], MOE["seed"] + 1000 * rank,
+                              pad_rows=0)
+    nbytes, flops = moe_algorithmic(mp)
+    names = ("m_indptr", "a", "b", "a_sf", "b_sf", "alpha", "d", "lora_b", "bias")
+    in_bytes = sum(getattr(mp, k).numel() * getattr(mp, k).element_size() for k in names)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(1, math.ceil(3 * l2 / in_bytes))
+    sets = [{k: getattr(mp, k).to(device) for k in names} for _ in range(copies)]
+    s = torch.tensor([MOE["lora_scale"]], dtype=torch.float32, device=device)
+    out = torch.empty((mp.rows, mp.N), dtype=torch.bfloat16, device=device)
+
+    def step(i):
+        t = sets[i % copies]
+        L.grouped_mm_nvfp4_lora(t["a"], t["b"], t["a_sf"], t["b_sf"], t["m_indptr"], t["alpha"], t["d"],
+                                t["lora_b"], s, bias=t["bias"], out=out)
+
+    steps = args.steps if args.steps is not None else WORKLOADS["moe"]["steps"]
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+        L.nvfp4lora_device_status(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(steps):
+                step(i)
+    upload_graph(g, stream)
+    g.replay()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        hold_device(stream)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    L.nvfp4lora_device_status(stream)
+    ms_total = e0.elapsed_time(e1)
+    if world > 1:
+        ms_total = max_over_ranks(ms_total, device)
+    ms = ms_total / steps
+    del g
+    value = flops / (ms * 1e-3) / 1e12
+    e2e = run_moe_e2e(L, mp, sets, s, device, min(steps, 200))
+    if world > 1:
+        e2e["ms_step"] = max_over_ranks(e2e["ms_step"], device)
+    roof = roofline_block(None, "moe", value, "TFLOPS", nbytes, ms_total)
+    line = {
+        "metric": METRIC, "value": whole_job(value, world), "unit": "TFLOPS", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3 -> fp32) + bf16 LoRA", "data": "synthetic",
+        "config": {"workload": f"moe: grouped call, {len(MOE['segments'])} experts with rows {list(MOE['segments'])}, "
+                               f"N={MOE['N']} K={MOE['K']} r={MOE['r']}, raw path + per-expert bias",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2_defeat": "inputs rotate through copies totalling >= 3x L2",
+                   "timing": "CUDA graph of K back-to-back calls (uploaded to the device before the timed region), "
+                             "CUDA events on the launching stream"},
+        "roofline": roof, "clocks": clk.summary(),
+        "e2e": {"value": whole_job(flops / (e2e["ms_step"] * 1e-3) / 1e12, world), "unit": "TFLOPS",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms_step"],
+                "steps": e2e["steps"],
+                "method": "grouped_mm_nvfp4_lora on device buffers filled from pinned host memory each step (a, a_sf, "
+                          "d, m_indptr), out copied back; two step slots on three streams, one CUDA graph"},
+        "gpu_launches": steps, "tflops": value, "gbs": nbytes / (ms * 1e-3) / 1e9, "weight_copies": copies,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, _ = moe_cpu_value(mp, 12.0)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOPS", "cores": oracle_threads(), "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_moe_e2e(L, mp, sets, s, device, steps):
+    """The grouped call end to end: each step copies the activation side (a, a_sf, d, m_indptr) host
+    -> device from pinned memory and out back; two step slots alternate over three streams."""
+    slots = 2
+    act = ("a", "a_sf", "d", "m_indptr")
+    host = [{k: getattr(mp, k).pin_memory() for k in act} for _ in range(slots)]
+    dev_in = [{k: torch.empty_like(getattr(mp, k), device=device) for k in act} for _ in range(slots)]
+    outs = [torch.empty((mp.rows, mp.N), dtype=torch.bfloat16, device=device) for _ in range(slots)]
+    outs_h = [torch.empty((mp.rows, mp.N), dtype=torch.bfloat16).pin_memory() for _ in range(slots)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    stream = torch.cuda.current_stream(device)
+    n_ev = steps + 8
+    ev_in = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_call = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_out = [torch.cuda.Event() for _ in range(n_ev)]
+    work = torch.cuda.Stream(device)
+
+    def one(i, first):
+        k = i % slots
+        with torch.cuda.stream(s_in):
+            if i - first >= slots:
+                s_in.wait_event(ev_call[i - slots])
+            for name in act:
+                dev_in[k][name].copy_(host[k][name], non_blocking=True)
+            ev_in[i].record(s_in)
+        with torch.cuda.stream(work):
+            work.wait_event(ev_in[i])
+            if i - first >= slots:
+                work.wait_event(ev_out[i - slots])
+            w = sets[i % len(sets)]
+            x = dev_in[k]
+            L.grouped_mm_nvfp4_lora(x["a"], w["b"], x["a_sf"], w["b_sf"], x["m_indptr"], w["alpha"], x["d"],
+                                    w["lora_b"], s, bias=w["bias"], out=outs[k])
+            ev_call[i].record(work)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_call[i])
+            outs_h[k].copy_(outs[k], non_blocking=True)
+            ev_out[i].record(s_out)
+
+    for i in range(4):
+        one(i, 0)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=work):
+        fork = torch.cuda.Event()
+        fork.record(work)
+        s_in.wait_event(fork)
+        s_out.wait_event(fork)
+        for i in range(steps):
+            one(i + 4, 4)
+        for st_ in (s_in, s_out):
+            join = torch.cuda.Event()
+            join.record(st_)
+            work.wait_event(join)
+    g.replay()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(work):
+        e0.record(work)
+        g.replay()
+        e1.record(work)
+    torch.cuda.synchronize(device)
+    L.nvfp4lora_device_status(work)
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    h2d = sum(getattr(mp, k).numel() * getattr(mp, k).element_size() for k in act)
+    return dict(ms_step=ms, steps=steps, h2d=h2d, d2h=mp.rows * mp.N * 2)
+
+
 def run_quant(args, rank, world, device):
     """The NVFP4 quantizer (fp4_quantize reading) on bf16 activations of cfg3's shape: HBM-bound,
     2 bytes read and 0.5 + 1/16 written per element.  Inputs rotate through copies totalling
@@ -918,6 +1123,8 @@ def run_reference(args, rank, world):
         return 0
     if args.workload == "quant":
         return run_reference_quant(args)
+    if args.workload == "moe":
+        return run_reference_moe(args)
     c = describe(args.workload)
     p = make_problem(c["M"], c["N"], c["K"], c["r"], c["seed"], alpha=c["alpha"],
                      lora_scale=c["lora_scale"], bias=c["bias"])
@@ -945,6 +1152,27 @@ def run_reference(args, rank, world):
                                    f"{ncols} of {c['N']} output columns "
                                    f"({sample_rows(c) * ncols / (c['M'] * c['N']):.5f} of the workload)"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_moe(args):
+    """Reference arm of the grouped workload: the oracle on a bounded sample per step."""
+    from workloads import MOE, make_grouped_problem
+    mp = make_grouped_problem(list(MOE["segments"]), MOE["N"], MOE["K"], MOE["r"], MOE["seed"], pad_rows=0)
+    K_steps = args.steps if args.steps is not None else 20
+    per_step = max(0.05, 120.0 / (K_steps + args.warmup))
+    value, sample, dt = moe_cpu_value(mp, per_step * K_steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": K_steps, "warmup": args.warmup, "ms_per_step": dt / K_steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"moe: grouped call, {len(MOE['segments'])} experts with rows {list(MOE['segments'])}, "
+                               f"N={MOE['N']} K={MOE['K']} r={MOE['r']}, raw path + per-expert bias"},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -1021,8 +1249,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", device_id=device,
                                              timeout=datetime.timedelta(seconds=120))
-    if args.workload in ("cfg4", "quant"):
-        rc = (run_cfg4 if args.workload == "cfg4" else run_quant)(args, rank, world, device)
+    if args.workload in ("cfg4", "quant", "moe"):
+        rc = {"cfg4": run_cfg4, "quant": run_quant, "moe": run_moe}[args.workload](args, rank, world, device)
         if world > 1:
             torch.distributed.destroy_process_group()
         return rc

@@ -143,6 +143,10 @@ CONFIGS = {
                  lora_scale=0.25, bias=False, seed=3),
 }
 
+#: grouped (expert-partitioned) layer: 8 experts with these row counts (multiples of 128, one
+#: empty), per-expert weights N x K, a shared rank-16 adapter scale, raw path with per-expert bias
+MOE = dict(segments=(512, 128, 1024, 256, 0, 384, 128, 640), N=4096, K=4096, r=16, lora_scale=0.5, seed=6)
+
 #: adapter-switch sweep: N=14336, K=4096, M x r grid, 8 adapters, alpha 2**-9
 CFG4 = dict(N=14336, K=4096, Ms=(1, 32, 256, 2048), rs=(8, 128), adapters=8,
             alpha=2.0 ** -9, seed=4)
