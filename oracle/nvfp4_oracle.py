@@ -19,6 +19,10 @@ It restates, slowly and in float64, what the pages define:
   ``b_folded[i] = bf16_rne(fp32(lora_b[i]) * ratio)``).
 * the quantizer the mm_nvfp4_lora page names as the producer of a / a_sf (``fp4_quantize``),
   by the reading given at :func:`quantize_nvfp4`.
+* ``flashinfer.grouped_mm.grouped_mm_bf16`` -- the grouped (expert-partitioned) form, by the
+  reading given at :func:`grouped_mm`.
+* ``flashinfer.fused_moe.bgmv_moe_gemm2_lora_delta`` -- opening formula and Parameters: the
+  routed-MoE FC2 LoRA delta, by the readings given at :func:`bgmv_moe_lora_delta`.
 
 Readings taken where the pages are silent:
 
@@ -459,6 +463,108 @@ def quantize_nvfp4(x_bits: np.ndarray, global_scale: float):
     codes = np.where((sfv > 0)[..., None], codes, np.uint8(0)).reshape(rows, k)
     packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
     return packed, swizzle_scales(sf, k, pad_value=0)
+
+
+# --------------------------------------------------------------------------------------
+# The routed-MoE FC2 LoRA delta (flashinfer.fused_moe.bgmv_moe_gemm2_lora_delta page: the
+# opening formula and Parameters).  For token t with adapter l = lora_ids[t] and routed slots j
+# (expert e = topk_ids[t, j], combine weight w = topk_weights[t, j], activation row
+# p = expanded_idx_to_permuted_idx[t * top_k + j]):
+#     delta[t] = scale * sum_j w * ( B_down[l, e] @ ( A_down[l, e] @ act[p] ) )
+# Readings taken where the page is silent:
+#   * A_down[l, e] is the [rank, I] row-major block that starts l * lora_stride_a elements into
+#     expert e's A bank (A_down @ act maps I -> rank); B_down[l, e] is the [H, rank] row-major
+#     block l * lora_stride_b elements into expert e's B bank (B_down @ v maps rank -> H);
+#   * the activation and both banks hold lora_dtype values (bf16 or fp16);
+#   * a token whose lora id is negative gets an all-zero delta; a slot whose permuted index is
+#     negative contributes nothing;
+#   * scale is taken as a float32 value; the delta is formed in float64 here (its error far below
+#     a float32 accumulation's) and rounded once to out_dtype (nearest, ties to even).
+# --------------------------------------------------------------------------------------
+
+def f16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """IEEE binary16 bit patterns -> float64 (exact)."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def f64_to_f16_rne(y: np.ndarray) -> np.ndarray:
+    """Round float64 straight to binary16 bits: nearest, ties to even, one rounding.
+
+    binary16 keeps 11 significant bits, normals down to 2**-14, subnormal quantum 2**-24 and a
+    largest finite value of 65504.  The quantum of |y| in [2**(E-1), 2**E) is
+    ``2**(max(E, -13) - 11)``; a rounded magnitude of 2**16 or more is infinity."""
+    y = np.asarray(y, dtype=np.float64)
+    sign = np.signbit(y)
+    mag = np.abs(y)
+    nz = np.isfinite(y) & (mag > 0)
+    _, exp = np.frexp(np.where(nz, mag, 1.0))
+    q = np.exp2((np.maximum(exp, -13) - 11).astype(np.float64))
+    rounded = np.rint(np.where(nz, mag, 0.0) / q) * q
+    overflow = nz & (rounded >= 2.0 ** 16)
+    out = np.where(overflow, 0.0, rounded).astype(np.float16).view(np.uint16).copy()
+    out[overflow | np.isinf(y)] = 0x7C00
+    out = np.where(sign, out | 0x8000, out).astype(np.uint16)
+    out[np.isnan(y)] = 0x7E00
+    return out
+
+
+def lora_values(bits, lora_dtype: str) -> np.ndarray:
+    """bf16 or fp16 bit patterns -> float64."""
+    if lora_dtype == "bf16":
+        return bf16_bits_to_f64(bits)
+    if lora_dtype == "fp16":
+        return f16_bits_to_f64(bits)
+    raise ValueError("lora_dtype must be 'bf16' or 'fp16'")
+
+
+def round_to(y: np.ndarray, out_dtype: str) -> np.ndarray:
+    """The single rounding of the delta to out_dtype (bf16 or fp16 bits)."""
+    if out_dtype == "bf16":
+        return f64_to_bf16_rne(y)
+    if out_dtype == "fp16":
+        return f64_to_f16_rne(y)
+    raise ValueError("out_dtype must be 'bf16' or 'fp16'")
+
+
+def bgmv_moe_lora_delta(act_bits, perm, a_banks, lora_stride_a: int, b_banks, lora_stride_b: int,
+                        topk_ids, topk_weights, lora_ids, rank: int, hidden_size: int, scale: float,
+                        lora_dtype: str = "bf16", tokens=None) -> np.ndarray:
+    """float64 delta rows [len(tokens) or T, H] before the output rounding.
+
+    act_bits: [padded_rows, I] bit patterns; perm: [T * top_k]; a_banks / b_banks: one flat bit
+    array per expert (the memory each pointer-table entry points at); topk_ids, topk_weights:
+    [T, top_k]; lora_ids: [T].  ``tokens`` selects the rows to evaluate (all when None)."""
+    act = lora_values(act_bits, lora_dtype)
+    rows, I = act.shape
+    ids = np.asarray(topk_ids, dtype=np.int64)
+    T, top_k = ids.shape
+    w = np.asarray(topk_weights, dtype=np.float32).astype(np.float64)
+    perm = np.asarray(perm, dtype=np.int64).reshape(T * top_k)
+    lids = np.asarray(lora_ids, dtype=np.int64).reshape(T)
+    s = float(np.float32(scale))
+    H = int(hidden_size)
+    sel = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64).reshape(-1)
+    out = np.zeros((sel.size, H), dtype=np.float64)
+    for i, t in enumerate(sel):
+        l = int(lids[t])
+        if l < 0:
+            continue
+        acc = np.zeros(H, dtype=np.float64)
+        for j in range(top_k):
+            p = int(perm[t * top_k + j])
+            if p < 0:
+                continue
+            if p >= rows:
+                raise ValueError("permuted index past the activation rows")
+            e = int(ids[t, j])
+            a0 = l * int(lora_stride_a)
+            b0 = l * int(lora_stride_b)
+            A = lora_values(np.asarray(a_banks[e]).reshape(-1)[a0:a0 + rank * I], lora_dtype).reshape(rank, I)
+            B = lora_values(np.asarray(b_banks[e]).reshape(-1)[b0:b0 + H * rank], lora_dtype).reshape(H, rank)
+            v = A @ act[p]                      # [rank]
+            acc += w[t, j] * (B @ v)            # [H]
+        out[i] = s * acc
+    return out
 
 
 # --------------------------------------------------------------------------------------

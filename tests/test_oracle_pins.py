@@ -584,3 +584,143 @@ def test_quantize_error_bound_random():
     back = O.dequant(packed, sf_buf, rows, k) / np.float32(gs)
     blk_amax = np.repeat(np.abs(xf).reshape(rows, k // 16, 16).max(axis=2), 16, axis=1)
     assert np.all(np.abs(back - xf) <= blk_amax / 6.0 * (1 + 2.0 ** -3))
+
+
+# ---------------------------------------------------------------------------------------
+# the routed-MoE FC2 LoRA delta (flashinfer.fused_moe.bgmv_moe_gemm2_lora_delta page)
+# ---------------------------------------------------------------------------------------
+
+def _half_closed_form(bits: int, dtype: str) -> float:
+    """bf16 / binary16 from the bit fields (bf16: 8 exponent bits, bias 127, 7 mantissa bits;
+    binary16: 5 exponent bits, bias 15, 10 mantissa bits); finite values only."""
+    eb, mb = (8, 7) if dtype == "bf16" else (5, 10)
+    bias = (1 << (eb - 1)) - 1
+    s = -1.0 if bits & 0x8000 else 1.0
+    e = (bits >> mb) & ((1 << eb) - 1)
+    m = bits & ((1 << mb) - 1)
+    assert e != (1 << eb) - 1
+    if e == 0:
+        return s * m * 2.0 ** (1 - bias - mb)
+    return s * (1.0 + m * 2.0 ** -mb) * 2.0 ** (e - bias)
+
+
+def _bits_of(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _bgmv_args(p, dtype: str):
+    return dict(act_bits=_bits_of(p.act), perm=p.perm.numpy(), a_banks=[_bits_of(x) for x in p.a_banks],
+                lora_stride_a=p.stride_a, b_banks=[_bits_of(x) for x in p.b_banks], lora_stride_b=p.stride_b,
+                topk_ids=p.topk_ids.numpy(), topk_weights=p.topk_weights.numpy(), lora_ids=p.lora_ids.numpy(),
+                rank=p.rank, hidden_size=p.H, scale=p.scale, lora_dtype=dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_bgmv_delta_against_a_brute_force_loop(dtype):
+    """Per element, in pure Python with the bit-field decoders: the page's sum over slots of
+    w * sum_k B[h, k] * sum_i A[k, i] * act[p, i], times scale; adapters addressed by stride
+    (with NaN padding between blocks, so a wrong offset shows), skipped tokens and slots."""
+    import workloads as W
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    p = W.make_bgmv_problem(6, 3, 4, 3, 16, 8, 8, seed=11, lora_dtype=tdt, scale=1.5, p_no_lora=0.2,
+                            p_inactive=0.2, stride_pad=8, seg_align=4)
+    p.topk_weights[2, 1] = -0.75                     # a negative combine weight
+    args = _bgmv_args(p, dtype)
+    got = O.bgmv_moe_lora_delta(**args)
+    act, ab, bb = args["act_bits"], args["a_banks"], args["b_banks"]
+    want = np.zeros((p.T, p.H))
+    for t in range(p.T):
+        l = int(p.lora_ids[t])
+        if l < 0:
+            continue
+        for h in range(p.H):
+            acc = 0.0
+            for j in range(p.top_k):
+                row = int(p.perm[t * p.top_k + j])
+                if row < 0:
+                    continue
+                e = int(p.topk_ids[t, j])
+                u = 0.0
+                for k in range(p.rank):
+                    v = 0.0
+                    for i in range(p.I):
+                        av = _half_closed_form(int(ab[e][l * p.stride_a + k * p.I + i]), dtype)
+                        v += av * _half_closed_form(int(act[row, i]), dtype)
+                    u += _half_closed_form(int(bb[e][l * p.stride_b + h * p.rank + k]), dtype) * v
+                acc += float(p.topk_weights[t, j]) * u
+            want[t, h] = float(np.float32(p.scale)) * acc
+    assert (p.lora_ids < 0).any() and (p.perm < 0).any()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-15)
+    rows = [1, 4]
+    np.testing.assert_array_equal(O.bgmv_moe_lora_delta(**args, tokens=rows), got[rows])
+
+
+def test_bgmv_single_route_is_two_library_matmuls():
+    """One token, one slot, weight 1, scale 1: B @ (A @ x) through PyTorch's float64 matmul."""
+    rng = np.random.default_rng(3)
+    I, H, r = 64, 48, 16
+    A = rng.standard_normal((r, I)); B = rng.standard_normal((H, r)); x = rng.standard_normal(I)
+    to_bits = lambda v: _bits_of(torch.tensor(v, dtype=torch.float32).to(torch.bfloat16))
+    Ab, Bb, xb = to_bits(A), to_bits(B), to_bits(x)
+    dec = lambda b: torch.tensor(b.astype(np.int16)).view(torch.bfloat16).double()
+    want = (dec(Bb).reshape(H, r) @ (dec(Ab).reshape(r, I) @ dec(xb))).numpy()
+    got = O.bgmv_moe_lora_delta(xb.reshape(1, I), [0], [Ab.reshape(-1)], r * I, [Bb.reshape(-1)], H * r,
+                                [[0]], [[1.0]], [0], r, H, 1.0)
+    np.testing.assert_allclose(got[0], want, rtol=1e-13, atol=1e-13)
+
+
+def test_bgmv_one_hot_fixes_adapter_expert_and_orientation():
+    """A single 1 at A[l*, e*][k0, i0] and B[l*, e*][h0, k0]: only out[t, h0] = scale * w * act[p, i0]
+    is non-zero, so a transposed A or B, a wrong adapter or expert offset, or a wrong activation
+    row moves or loses it."""
+    I, H, r, E, L = 32, 24, 8, 3, 4
+    l0, e0, k0, i0, h0 = 2, 1, 5, 17, 19
+    a_banks = [np.zeros(L * r * I, dtype=np.uint16) for _ in range(E)]
+    b_banks = [np.zeros(L * H * r, dtype=np.uint16) for _ in range(E)]
+    one = 0x3F80                                       # bf16 1.0
+    a_banks[e0][l0 * r * I + k0 * I + i0] = one
+    b_banks[e0][l0 * H * r + h0 * r + k0] = one
+    act = np.zeros((4, I), dtype=np.uint16)
+    act[3, i0] = 0x4040                                # 3.0
+    act[2, i0] = 0x4100                                # 8.0 (a row no slot of token 1 uses)
+    got = O.bgmv_moe_lora_delta(act, [2, 0, 3, 1], a_banks, r * I, b_banks, H * r,
+                                [[0, 2], [1, 0]], [[0.5, 0.5], [0.25, 0.75]], [l0, l0], r, H, 2.0)
+    want = np.zeros((2, H))
+    want[1, h0] = 2.0 * 0.25 * 3.0
+    np.testing.assert_array_equal(got, want)
+
+
+def test_bgmv_invariants_slot_order_inactive_slots_and_no_adapter():
+    import workloads as W
+    p = W.make_bgmv_problem(8, 3, 5, 2, 32, 16, 8, seed=5, p_no_lora=0.25, p_inactive=0.0, seg_align=8)
+    args = _bgmv_args(p, "bf16")
+    base = O.bgmv_moe_lora_delta(**args)
+    # the slots of a token may come in any order
+    order = [2, 0, 1]
+    args2 = dict(args, topk_ids=p.topk_ids.numpy()[:, order], topk_weights=p.topk_weights.numpy()[:, order],
+                 perm=p.perm.numpy().reshape(p.T, 3)[:, order].reshape(-1))
+    np.testing.assert_allclose(O.bgmv_moe_lora_delta(**args2), base, rtol=1e-12, atol=1e-15)
+    # an inactive slot equals a problem without that slot
+    perm3 = p.perm.numpy().copy().reshape(p.T, 3)
+    perm3[:, 2] = -1
+    args3 = dict(args, perm=perm3.reshape(-1))
+    args4 = dict(args, topk_ids=p.topk_ids.numpy()[:, :2], topk_weights=p.topk_weights.numpy()[:, :2],
+                 perm=p.perm.numpy().reshape(p.T, 3)[:, :2].reshape(-1))
+    np.testing.assert_allclose(O.bgmv_moe_lora_delta(**args3), O.bgmv_moe_lora_delta(**args4), rtol=1e-12)
+    # no adapter: zero row; linear in scale
+    assert np.all(base[p.lora_ids.numpy() < 0] == 0) and (p.lora_ids < 0).any()
+    np.testing.assert_allclose(O.bgmv_moe_lora_delta(**dict(args, scale=2 * p.scale)), 2 * base, rtol=1e-15)
+
+
+def test_f16_rounding_against_numpy_and_hand_cases():
+    rng = np.random.default_rng(2)
+    y = np.concatenate([rng.standard_normal(20000) * np.exp2(rng.integers(-30, 17, 20000)),
+                        [1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 2.0 ** -25, 3 * 2.0 ** -26, 65519.99, 65520.0,
+                         -65520.0, 2.0 ** -24 * 0.5, 0.0, -0.0]])
+    got = O.f64_to_f16_rne(y)
+    with np.errstate(over="ignore"):
+        want = y.astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(got, want)
+    assert got[-10] == 0x3C00 and got[-9] == 0x3C02          # ties to even at 1
+    assert got[-6] == 0x7BFF and got[-5] == 0x7C00 and got[-4] == 0xFC00
+    assert got[-3] == 0x0000 and got[-1] == 0x8000             # half the smallest subnormal -> 0

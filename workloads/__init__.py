@@ -126,6 +126,78 @@ def make_adapters(N: int, r: int, count: int, seed: int, lb_std: float = 0.02):
     return out
 
 
+@dataclasses.dataclass
+class BgmvProblem:
+    """One routed-MoE LoRA-delta problem's host tensors (CPU, contiguous)."""
+    T: int
+    top_k: int
+    num_experts: int
+    num_adapters: int
+    I: int
+    H: int
+    rank: int
+    lora_dtype: torch.dtype
+    scale: float
+    act: torch.Tensor            # lora_dtype [padded_rows, I], permuted rows
+    perm: torch.Tensor           # int32 [T * top_k]: expanded index -> permuted row, -1 inactive
+    a_banks: list                # per expert: lora_dtype [num_adapters * stride_a]
+    stride_a: int
+    b_banks: list                # per expert: lora_dtype [num_adapters * stride_b]
+    stride_b: int
+    topk_ids: torch.Tensor       # int32 [T, top_k], distinct experts per token
+    topk_weights: torch.Tensor   # fp32 [T, top_k], positive, summing to 1 per token
+    lora_ids: torch.Tensor       # int32 [T], -1 = no adapter
+
+
+def make_bgmv_problem(T: int, top_k: int, num_experts: int, num_adapters: int, I: int, H: int,
+                      rank: int, seed: int, *, lora_dtype=torch.bfloat16, scale: float = 2.0,
+                      p_no_lora: float = 0.125, p_inactive: float = 0.0625, stride_pad: int = 0,
+                      act_std: float = 0.5, b_std: float = 0.02, seg_align: int = 128) -> BgmvProblem:
+    """Draw one problem.  Routing: each token picks top_k distinct experts (a random permutation
+    per token) with softmax weights of N(0, 1) logits; the expanded slots are laid out grouped by
+    expert, each expert's segment padded to a multiple of `seg_align` rows, as a grouped FC1
+    would return them; a fraction `p_inactive` of slots is marked inactive (-1) and a fraction
+    `p_no_lora` of tokens gets lora id -1.  A_down ~ U(-1/sqrt(I), 1/sqrt(I)), B_down ~ N(0,
+    b_std), activations ~ N(0, act_std).  Each adapter block is followed by `stride_pad` NaN
+    elements (so a read outside a block shows).  Draw order: routing, weights, inactive slots,
+    lora ids, act, A banks, B banks."""
+    g = torch.Generator().manual_seed(seed)
+    ids = torch.stack([torch.randperm(num_experts, generator=g)[:top_k] for _ in range(T)]) if T else \
+        torch.zeros(0, top_k, dtype=torch.int64)
+    logits = torch.randn(T, top_k, generator=g)
+    w = torch.softmax(logits, dim=1).to(torch.float32)
+    inactive = torch.rand(T * top_k, generator=g) < p_inactive
+    no_lora = torch.rand(T, generator=g) < p_no_lora
+    lora_ids = torch.randint(0, num_adapters, (T,), generator=g, dtype=torch.int32)
+    lora_ids[no_lora] = -1
+    # slot layout: grouped by expert (slot order within an expert by expanded index)
+    flat = ids.reshape(-1)
+    perm = torch.full((T * top_k,), -1, dtype=torch.int32)
+    row = 0
+    for e in range(num_experts):
+        slots = (flat == e).nonzero().reshape(-1)
+        for n, x in enumerate(slots.tolist()):
+            perm[x] = row + n
+        row += -(-slots.numel() // seg_align) * seg_align
+    perm[inactive] = -1
+    padded_rows = max(row, seg_align)
+    act = (torch.randn(padded_rows, I, generator=g) * act_std).to(lora_dtype)
+    stride_a = rank * I + stride_pad
+    stride_b = H * rank + stride_pad
+    bound = 1.0 / (I ** 0.5)
+    a_banks, b_banks = [], []
+    for _ in range(num_experts):
+        bank = torch.full((num_adapters, stride_a), float("nan"))
+        bank[:, :rank * I] = torch.empty(num_adapters, rank * I).uniform_(-bound, bound, generator=g)
+        a_banks.append(bank.reshape(-1).to(lora_dtype))
+    for _ in range(num_experts):
+        bank = torch.full((num_adapters, stride_b), float("nan"))
+        bank[:, :H * rank] = torch.randn(num_adapters, H * rank, generator=g) * b_std
+        b_banks.append(bank.reshape(-1).to(lora_dtype))
+    return BgmvProblem(T, top_k, num_experts, num_adapters, I, H, rank, lora_dtype, float(scale), act, perm,
+                       a_banks, stride_a, b_banks, stride_b, ids.to(torch.int32), w, lora_ids)
+
+
 # --------------------------------------------------------------------------------------
 # The workloads (shapes, paths and scalars).  "cfg0" is the small parity case; "cfg1" is
 # the decode shape the throughput metric is quoted on at M <= 16; "cfg2"/"cfg3" are the
@@ -146,6 +218,11 @@ CONFIGS = {
 #: grouped (expert-partitioned) layer: 8 experts with these row counts (multiples of 128, one
 #: empty), per-expert weights N x K, a shared rank-16 adapter scale, raw path with per-expert bias
 MOE = dict(segments=(512, 128, 1024, 256, 0, 384, 128, 640), N=4096, K=4096, r=16, lora_scale=0.5, seed=6)
+
+#: routed-MoE FC2 LoRA delta: a decode batch of 64 tokens routed top-2 over the layer's 8 experts,
+#: I = H = 4096 (the layer's width), rank 16, 4 adapters, scale 2 (an assumed serving mix; the
+#: pages give no shapes for it)
+BGMV = dict(T=64, top_k=2, num_experts=8, num_adapters=4, I=4096, H=4096, rank=16, scale=2.0, seed=7)
 
 #: adapter-switch sweep: N=14336, K=4096, M x r grid, 8 adapters, alpha 2**-9
 CFG4 = dict(N=14336, K=4096, Ms=(1, 32, 256, 2048), rs=(8, 128), adapters=8,
