@@ -45,6 +45,7 @@ WORKLOADS = {
     "cfg4": dict(src=None, steps=None),   # adapter-switch sweep (its own runner)
     "quant": dict(src=None, steps=400),   # the NVFP4 quantizer on the cfg3 activations (its own runner)
     "moe": dict(src=None, steps=200),     # the grouped call on an 8-expert layer (its own runner)
+    "bgmv": dict(src=None, steps=2000),   # the routed-MoE FC2 LoRA delta on a decode batch (its own runner)
 }
 
 QUANT_ROWS, QUANT_K = 8192, 8192         # cfg3's a: M x K
@@ -170,13 +171,15 @@ def measured_peaks():
 def source_hash(kernel="gemm"):
     """Hash of the kernel sources a recorded ncu figure depends on: the GEMM kernels (tiled, SM-pair,
     decode), the fold and the PTX wrappers for `gemm`, the quantizer and the wrappers for
-    `quantize`.  The host launcher is not hashed: a change of a launch configuration there is
+    `quantize`, the LoRA-delta kernel and the headers it includes for `bgmv_delta`.  The host launcher is not hashed: a change of a launch configuration there is
     re-captured by hand."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "nvfp4_block_scaled_mm_b200", "csrc")
     if kernel == "quantize":
         files = ["ptx.cuh", "quantize.cuh"]
+    elif kernel == "bgmv_delta":
+        files = ["bgmv.cuh", "fold.cuh", "ptx.cuh"]
     else:
         files = ["fold.cuh", "gemm.cuh", "gemm_decode.cuh", "gemm_pair.cuh", "ptx.cuh"]
     for f in files:
@@ -771,6 +774,231 @@ def run_moe_e2e(L, mp, sets, s, device, steps):
     return dict(ms_step=ms, steps=steps, h2d=h2d, d2h=mp.rows * mp.N * 2)
 
 
+def bgmv_workload_text():
+    from workloads import BGMV
+    return (f"bgmv: routed-MoE FC2 LoRA delta, T={BGMV['T']} tokens top-{BGMV['top_k']} of {BGMV['num_experts']} "
+            f"experts, {BGMV['num_adapters']} adapters, I={BGMV['I']} H={BGMV['H']} rank={BGMV['rank']}, bf16")
+
+
+def bgmv_algorithmic(bp):
+    """Algorithmic bytes and flops of one delta call: the active slots' activation rows, every
+    (adapter, expert) block pair that an active slot uses (A and B once each), the routing and
+    pointer tables, and the output."""
+    ids = bp.topk_ids.numpy()
+    perm = bp.perm.numpy().reshape(bp.T, bp.top_k)
+    lids = bp.lora_ids.numpy()
+    pairs, rows = set(), 0
+    for t in range(bp.T):
+        if lids[t] < 0:
+            continue
+        for j in range(bp.top_k):
+            if perm[t, j] >= 0:
+                rows += 1
+                pairs.add((int(lids[t]), int(ids[t, j])))
+    el = 2
+    nbytes = (rows * bp.I * el + len(pairs) * (bp.rank * bp.I + bp.H * bp.rank) * el + bp.T * bp.top_k * 12
+              + bp.T * 4 + 2 * bp.num_experts * 8 + bp.T * bp.H * el)
+    return nbytes, 2 * rows * (bp.rank * bp.I + bp.H * bp.rank)
+
+
+def bgmv_cpu_value(bp, budget_s):
+    """Oracle throughput (GB/s of the call's algorithmic bytes) on bounded token samples."""
+    import oracle as O
+    nbytes, _ = bgmv_algorithmic(bp)
+    b16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    act, ab, bb = b16(bp.act), [b16(x) for x in bp.a_banks], [b16(x) for x in bp.b_banks]
+    ntok = 8
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        toks = np.arange(reps * ntok, (reps + 1) * ntok) % bp.T
+        O.round_to(O.bgmv_moe_lora_delta(act, bp.perm.numpy(), ab, bp.stride_a, bb, bp.stride_b,
+                                         bp.topk_ids.numpy(), bp.topk_weights.numpy(), bp.lora_ids.numpy(),
+                                         bp.rank, bp.H, bp.scale, "bf16", tokens=toks), "bf16")
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s or reps >= 400:
+            break
+    dt = time.perf_counter() - t0
+    frac = reps * ntok / bp.T
+    return nbytes * frac / dt / 1e9, f"{reps} x oracle delta on {ntok} of {bp.T} tokens, {dt:.1f} s", dt
+
+
+def run_bgmv(args, rank, world, device):
+    """The routed-MoE FC2 LoRA delta on a decode batch (workloads.BGMV): memory-bound, reported in
+    GB/s of algorithmic bytes against the measured HBM copy bandwidth.  Activations, banks and
+    routing rotate through copies totalling >= 3x L2; K calls in one CUDA graph."""
+    import nvfp4_block_scaled_mm_b200 as L
+    from workloads import BGMV, make_bgmv_problem
+    cfg = dict(BGMV)
+    cfg["seed"] = BGMV["seed"] + 1000 * rank
+    bp = make_bgmv_problem(**cfg)
+    nbytes, flops = bgmv_algorithmic(bp)
+    route = ("perm", "topk_ids", "topk_weights", "lora_ids")
+    in_bytes = (bp.act.numel() * 2 + sum(x.numel() * 2 for x in bp.a_banks + bp.b_banks)
+                + sum(getattr(bp, k).numel() * 4 for k in route))
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(1, math.ceil(3 * l2 / in_bytes))
+    sets = []
+    for _ in range(copies):
+        a = [x.to(device) for x in bp.a_banks]
+        b = [x.to(device) for x in bp.b_banks]
+        sets.append(dict(act=bp.act.to(device), a=a, b=b, wa=L.fill_w_ptr(a), wb=L.fill_w_ptr(b),
+                         **{k: getattr(bp, k).to(device) for k in route}))
+    out = torch.empty((bp.T, bp.H), dtype=torch.bfloat16, device=device)
+
+    def call(t, act, o):
+        L.bgmv_moe_gemm2_lora_delta(act, t["perm"], t["wa"], bp.stride_a, t["wb"], bp.stride_b, t["topk_ids"],
+                                    t["topk_weights"], t["lora_ids"], bp.rank, bp.H, scale=bp.scale, out=o)
+
+    steps = args.steps if args.steps is not None else WORKLOADS["bgmv"]["steps"]
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            call(sets[i % copies], sets[i % copies]["act"], out)
+        L.nvfp4lora_device_status(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(steps):
+                call(sets[i % copies], sets[i % copies]["act"], out)
+    upload_graph(g, stream)
+    g.replay()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        hold_device(stream)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    L.nvfp4lora_device_status(stream)
+    ms_total = e0.elapsed_time(e1)
+    if world > 1:
+        ms_total = max_over_ranks(ms_total, device)
+    ms = ms_total / steps
+    del g
+    value = nbytes / (ms * 1e-3) / 1e9
+
+    # end to end: the activation rows and the routing tables come from pinned host memory every step,
+    # the delta goes back; the adapter banks stay resident (model state)
+    slots = 4
+    host = [dict(act=bp.act.pin_memory(), **{k: getattr(bp, k).pin_memory() for k in route}) for _ in range(slots)]
+    dev_in = [{k: torch.empty_like(v, device=device) for k, v in h.items()} for h in host]
+    outs = [torch.empty((bp.T, bp.H), dtype=torch.bfloat16, device=device) for _ in range(slots)]
+    outs_h = [torch.empty((bp.T, bp.H), dtype=torch.bfloat16).pin_memory() for _ in range(slots)]
+    s_in, s_out, work = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
+    e2e_steps = min(steps, 2000)
+    n_ev = e2e_steps + 8
+    ev_in = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_call = [torch.cuda.Event() for _ in range(n_ev)]
+    ev_out = [torch.cuda.Event() for _ in range(n_ev)]
+
+    def one(i, first):
+        k = i % slots
+        with torch.cuda.stream(s_in):
+            if i - first >= slots:
+                s_in.wait_event(ev_call[i - slots])
+            for name, h in host[k].items():
+                dev_in[k][name].copy_(h, non_blocking=True)
+            ev_in[i].record(s_in)
+        with torch.cuda.stream(work):
+            work.wait_event(ev_in[i])
+            if i - first >= slots:
+                work.wait_event(ev_out[i - slots])
+            w = dict(sets[i % copies])
+            w.update({name: dev_in[k][name] for name in route})
+            call(w, dev_in[k]["act"], outs[k])
+            ev_call[i].record(work)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_call[i])
+            outs_h[k].copy_(outs[k], non_blocking=True)
+            ev_out[i].record(s_out)
+
+    for i in range(4):
+        one(i, 0)
+    torch.cuda.synchronize(device)
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=work):
+        fork = torch.cuda.Event()
+        fork.record(work)
+        s_in.wait_event(fork)
+        s_out.wait_event(fork)
+        for i in range(e2e_steps):
+            one(i + 4, 4)
+        for st_ in (s_in, s_out):
+            join = torch.cuda.Event()
+            join.record(st_)
+            work.wait_event(join)
+    ge.replay()
+    torch.cuda.synchronize(device)
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(work):
+        e2.record(work)
+        ge.replay()
+        e3.record(work)
+    torch.cuda.synchronize(device)
+    L.nvfp4lora_device_status(work)
+    ms_e2e = e2.elapsed_time(e3) / e2e_steps
+    del ge
+    if world > 1:
+        ms_e2e = max_over_ranks(ms_e2e, device)
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+
+    roof = roofline_block(None, "bgmv", value, "GB/s", nbytes, ms_total)
+    roof["traffic"] = recorded_traffic("bgmv", "bgmv_delta")
+    line = {
+        "metric": METRIC, "value": whole_job(value, world), "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 x bf16 -> fp32", "data": "synthetic",
+        "config": {"workload": bgmv_workload_text(),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2_defeat": "activations, banks and routing rotate through copies totalling >= 3x L2",
+                   "timing": "CUDA graph of K back-to-back calls (uploaded to the device before the timed region), "
+                             "CUDA events on the launching stream"},
+        "roofline": roof, "clocks": clk.summary(),
+        "e2e": {"value": whole_job(nbytes / (ms_e2e * 1e-3) / 1e9, world), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": bp.T * bp.H * 2, "ms_per_step": ms_e2e,
+                "steps": e2e_steps,
+                "method": "bgmv_moe_gemm2_lora_delta with the activation rows and routing tables copied from pinned "
+                          "host memory each step and the delta copied back; banks resident; four step slots on "
+                          "three streams, one CUDA graph"},
+        "gpu_launches": steps, "gflops": flops / (ms * 1e-3) / 1e9, "copies": copies,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, _ = bgmv_cpu_value(bp, 10.0)
+        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_bgmv(args):
+    """Reference arm of the LoRA-delta workload: the oracle on a bounded token sample per step."""
+    from workloads import BGMV, make_bgmv_problem
+    bp = make_bgmv_problem(**BGMV)
+    K_steps = args.steps if args.steps is not None else 20
+    per_step = max(0.05, 120.0 / (K_steps + args.warmup))
+    value, sample, dt = bgmv_cpu_value(bp, per_step * K_steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": K_steps, "warmup": args.warmup, "ms_per_step": dt / K_steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": bgmv_workload_text()},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_quant(args, rank, world, device):
     """The NVFP4 quantizer (fp4_quantize reading) on bf16 activations of cfg3's shape: HBM-bound,
     2 bytes read and 0.5 + 1/16 written per element.  Inputs rotate through copies totalling
@@ -1125,6 +1353,8 @@ def run_reference(args, rank, world):
         return run_reference_quant(args)
     if args.workload == "moe":
         return run_reference_moe(args)
+    if args.workload == "bgmv":
+        return run_reference_bgmv(args)
     c = describe(args.workload)
     p = make_problem(c["M"], c["N"], c["K"], c["r"], c["seed"], alpha=c["alpha"],
                      lora_scale=c["lora_scale"], bias=c["bias"])
@@ -1249,8 +1479,9 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", device_id=device,
                                              timeout=datetime.timedelta(seconds=120))
-    if args.workload in ("cfg4", "quant", "moe"):
-        rc = {"cfg4": run_cfg4, "quant": run_quant, "moe": run_moe}[args.workload](args, rank, world, device)
+    if args.workload in ("cfg4", "quant", "moe", "bgmv"):
+        rc = {"cfg4": run_cfg4, "quant": run_quant, "moe": run_moe, "bgmv": run_bgmv}[args.workload](
+            args, rank, world, device)
         if world > 1:
             torch.distributed.destroy_process_group()
         return rc

@@ -200,8 +200,10 @@ NVFP4LORA_API nvfp4lora_status nvfp4lora_grouped_mm(
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error word that
- * kernels set when one of their bounded waits runs out.  Returns NVFP4LORA_OK or
- * NVFP4LORA_ERR_DEVICE_TIMEOUT (or NVFP4LORA_ERR_CUDA).
+ * kernels set when one of their bounded waits runs out (NVFP4LORA_ERR_DEVICE_TIMEOUT) or
+ * when a table read on the device breaks its rules (a grouped call's m_indptr, a LoRA delta's
+ * routing: NVFP4LORA_ERR_INVALID_ARG).  Returns NVFP4LORA_OK when the word was clear (or
+ * NVFP4LORA_ERR_CUDA).
  * The GEMM, fold and quantize calls return NVFP4LORA_OK once their work is enqueued; a kernel
  * whose bounded wait gives up returns early and leaves its outputs (out, b_folded, ratio, codes,
  * scales) partly unwritten.  Their contents are therefore defined only once a later
@@ -242,6 +244,52 @@ NVFP4LORA_API nvfp4lora_status nvfp4lora_quantize(
     const uint16_t* x, int64_t rows, int64_t K, const float* global_scale,
     uint8_t* codes, uint8_t* scales, int64_t scales_bytes,
     nvfp4lora_stream stream);
+
+/* Element types of the routed-MoE LoRA delta's activation, banks and output. */
+typedef enum nvfp4lora_dtype {
+    NVFP4LORA_DTYPE_BF16 = 0,
+    NVFP4LORA_DTYPE_FP16 = 1
+} nvfp4lora_dtype;
+
+/*
+ * Routed-MoE FC2 (down projection) LoRA delta: flashinfer.fused_moe.bgmv_moe_gemm2_lora_delta
+ * (opening formula and Parameters).  For every token t with adapter l = lora_ids[t]:
+ *     out[t] = scale * sum_j topk_weights[t, j] * ( B_down[l, e] @ ( A_down[l, e] @ act[p] ) )
+ * over its routed slots j (e = topk_ids[t, j], p = expanded_idx_to_permuted_idx[t*top_k + j]),
+ * to be added to the MoE output by the caller.  Readings taken where the page is silent:
+ * A_down[l, e] is the [rank, I] row-major block that starts l*lora_stride_a elements after
+ * w_ptr_a[e]; B_down[l, e] the [H, rank] row-major block l*lora_stride_b elements after
+ * w_ptr_b[e]; act and both banks hold lora_dtype values; a negative lora id gives an all-zero
+ * row; a negative permuted index is an inactive slot; the sum is formed in fp32 and rounded once
+ * to out_dtype (nearest, ties to even).
+ *   act      lora_dtype [padded_rows, I] device, row-major, 16-byte aligned (the permuted
+ *            post-activation rows of the MoE's first GEMM).  I % 8 == 0.
+ *   expanded_idx_to_permuted_idx  int32 [num_tokens * top_k] device.
+ *   w_ptr_a, w_ptr_b  int64 [num_experts] device tables of bank addresses (device memory of
+ *            this GPU, caller-owned and alive until the call completes); a bank address plus
+ *            l * stride * 2 bytes must be 16-byte aligned, so lora_stride_a % 8 == 0 and
+ *            lora_stride_b % 8 == 0.  Adapter ids must index adapters that exist in the banks:
+ *            the library cannot see the banks' sizes.
+ *   topk_ids int32 [num_tokens, top_k]; topk_weights fp32 [num_tokens, top_k];
+ *   lora_ids int32 [num_tokens]; all device.
+ *   rank     8 <= rank <= 128, rank % 8 == 0.   1 <= top_k <= 16.   hidden_size = H >= 1.
+ *   out      out_dtype [num_tokens, H] device, caller-owned, fully written.
+ * Every rule above that the host can see is checked before any CUDA call
+ * (NVFP4LORA_ERR_INVALID_ARG, nothing enqueued).  Routing entries are read on the device: an
+ * expert id outside [0, num_experts), a permuted index >= padded_rows or a bank address that
+ * is null or misaligned is skipped, and the next nvfp4lora_device_status returns
+ * NVFP4LORA_ERR_INVALID_ARG.  num_tokens == 0 enqueues nothing.  Enqueued on `stream`.
+ */
+NVFP4LORA_API nvfp4lora_status nvfp4lora_bgmv_moe_gemm2_lora_delta(
+    const void* act, int64_t padded_rows, int64_t I,
+    const int32_t* expanded_idx_to_permuted_idx,
+    const int64_t* w_ptr_a, int64_t lora_stride_a,
+    const int64_t* w_ptr_b, int64_t lora_stride_b,
+    const int32_t* topk_ids, const float* topk_weights, const int32_t* lora_ids,
+    int64_t num_tokens, int64_t top_k, int64_t num_experts,
+    int64_t rank, int64_t hidden_size,
+    int32_t lora_dtype, float scale, int32_t out_dtype,
+    void* out, nvfp4lora_stream stream);
 
 /* Message of the last failing call on this host thread ("" when none). */
 NVFP4LORA_API const char* nvfp4lora_last_error(void);

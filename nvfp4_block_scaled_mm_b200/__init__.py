@@ -14,7 +14,9 @@ Two layers:
   status mapped to exceptions);
 * ``mm_nvfp4_lora``, ``prepare_nvfp4_lora_adapter``, ``PreparedNvFp4LoraAdapter``,
   ``StaleAdapterError`` -- the API of flashinfer.gemm.mm_nvfp4_lora and
-  flashinfer.gemm.prepare_nvfp4_lora_adapter (signatures, Parameters, Returns, Notes).
+  flashinfer.gemm.prepare_nvfp4_lora_adapter (signatures, Parameters, Returns, Notes);
+  ``grouped_mm_nvfp4_lora`` (grouped_mm_bf16's grouped form), ``fp4_quantize``, and
+  ``bgmv_moe_gemm2_lora_delta`` / ``fill_w_ptr`` (flashinfer.fused_moe.bgmv_moe_gemm2_lora_delta).
 """
 
 from __future__ import annotations
@@ -31,7 +33,8 @@ __all__ = [
     "StaleAdapterError", "PreparedNvFp4LoraAdapter", "mm_nvfp4_lora", "prepare_nvfp4_lora_adapter",
     "nvfp4lora_mm", "nvfp4lora_prepare", "nvfp4lora_refold", "nvfp4lora_mm_prepared",
     "nvfp4lora_device_status", "nvfp4lora_quantize", "fp4_quantize", "library_path", "version",
-    "nvfp4lora_grouped_mm", "grouped_mm_nvfp4_lora",
+    "nvfp4lora_grouped_mm", "grouped_mm_nvfp4_lora", "nvfp4lora_bgmv_moe_gemm2_lora_delta",
+    "bgmv_moe_gemm2_lora_delta", "fill_w_ptr",
 ]
 
 OK, INVALID_ARG, STALE, ALPHA_ZERO, UNSUPPORTED_ARCH, DEVICE_TIMEOUT, CUDA_ERR = range(7)
@@ -68,6 +71,9 @@ def _load():
     lib.nvfp4lora_quantize.restype = ctypes.c_int
     lib.nvfp4lora_grouped_mm.argtypes = [P, P, P, I64, P, I64, P, I64, P, P, P, P, I64, P, P, I64, I64, I64, P]
     lib.nvfp4lora_grouped_mm.restype = ctypes.c_int
+    lib.nvfp4lora_bgmv_moe_gemm2_lora_delta.argtypes = [P, I64, I64, P, P, I64, P, I64, P, P, P, I64, I64, I64, I64,
+                                                        I64, ctypes.c_int32, ctypes.c_float, ctypes.c_int32, P, P]
+    lib.nvfp4lora_bgmv_moe_gemm2_lora_delta.restype = ctypes.c_int
     lib.nvfp4lora_last_error.argtypes = []
     lib.nvfp4lora_last_error.restype = ctypes.c_char_p
     lib.nvfp4lora_version.argtypes = []
@@ -181,8 +187,20 @@ def nvfp4lora_grouped_mm(a, b, a_sf, b_sf, m_indptr, num_experts, alpha, d, lora
     return out
 
 
+def nvfp4lora_bgmv_moe_gemm2_lora_delta(act, padded_rows, I, perm, w_ptr_a, lora_stride_a, w_ptr_b, lora_stride_b,
+                                        topk_ids, topk_weights, lora_ids, num_tokens, top_k, num_experts, rank,
+                                        hidden_size, lora_dtype, scale, out_dtype, out, stream=None):
+    _check(_lib.nvfp4lora_bgmv_moe_gemm2_lora_delta(
+        _ptr(act), int(padded_rows), int(I), _ptr(perm), _ptr(w_ptr_a), int(lora_stride_a), _ptr(w_ptr_b),
+        int(lora_stride_b), _ptr(topk_ids), _ptr(topk_weights), _ptr(lora_ids), int(num_tokens), int(top_k),
+        int(num_experts), int(rank), int(hidden_size), int(lora_dtype), float(scale), int(out_dtype), _ptr(out),
+        _stream(stream)))
+    return out
+
+
 def nvfp4lora_device_status(stream=None) -> None:
-    """Synchronise the stream and raise DeviceTimeoutError if a kernel's wait ran out."""
+    """Synchronise the stream; raise DeviceTimeoutError if a kernel's wait ran out, ValueError if a
+    table read on the device (a grouped call's m_indptr, a LoRA delta's routing) broke its rules."""
     _check(_lib.nvfp4lora_device_status(_stream(stream)))
 
 
@@ -419,6 +437,85 @@ def grouped_mm_nvfp4_lora(a: torch.Tensor, b: torch.Tensor, a_sf: torch.Tensor, 
         nvfp4lora_grouped_mm(a, b, a_sf, b_sf, m_indptr, E, alpha, d if lora_scale is not None else None,
                              lora_b if lora_scale is not None else None, lora_scale, r, bias, out, rows, N, K,
                              torch.cuda.current_stream(a.device))
+    return out
+
+
+_DTYPE_CODES = {torch.bfloat16: 0, torch.float16: 1}
+
+
+def fill_w_ptr(banks) -> torch.Tensor:
+    """The int64 ``[1, num_experts]`` table of bank addresses that
+    :func:`bgmv_moe_gemm2_lora_delta` takes as ``w_ptr_a`` / ``w_ptr_b``: entry e is the device
+    address of ``banks[e]`` (one contiguous bf16 or fp16 CUDA tensor per expert, holding that
+    expert's adapters ``lora_stride`` elements apart).  The table does not keep the banks alive."""
+    banks = list(banks)
+    if not banks:
+        raise ValueError("fill_w_ptr needs at least one bank")
+    dev = banks[0].device
+    for i, t in enumerate(banks):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"bank {i} must be a contiguous CUDA tensor")
+        if t.dtype not in _DTYPE_CODES:
+            raise ValueError(f"bank {i} must be bf16 or fp16, got {t.dtype}")
+        if t.device != dev:
+            raise ValueError(f"bank {i} is on {t.device} but bank 0 is on {dev}")
+    return torch.tensor([[t.data_ptr() for t in banks]], dtype=torch.int64, device=dev)
+
+
+def bgmv_moe_gemm2_lora_delta(gemm1_activation_output: torch.Tensor, expanded_idx_to_permuted_idx: torch.Tensor,
+                              w_ptr_a: torch.Tensor, lora_stride_a: int, w_ptr_b: torch.Tensor,
+                              lora_stride_b: int, topk_ids: torch.Tensor, topk_weights: torch.Tensor,
+                              lora_ids: torch.Tensor, rank: int, hidden_size: int, *,
+                              lora_dtype: torch.dtype = torch.bfloat16, scale: float = 1.0,
+                              out_dtype: torch.dtype = torch.bfloat16,
+                              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """FC2 (down projection) LoRA delta of a routed MoE, flashinfer.fused_moe.bgmv_moe_gemm2_lora_delta:
+    ``delta[t] = scale * sum_j topk_weights[t, j] * (B_down[l, e] @ (A_down[l, e] @ act[p]))`` with
+    ``l = lora_ids[t]`` (negative: a zero row), ``e = topk_ids[t, j]`` and
+    ``p = expanded_idx_to_permuted_idx[t * top_k + j]`` (negative: inactive slot).  Returns
+    ``[T, hidden_size]`` in out_dtype, to be added to the MoE output.
+
+    gemm1_activation_output: lora_dtype ``[padded_rows, I]`` (I % 8 == 0); the index, id and weight
+    tensors are int32 / int32 / fp32 as shaped on the page; ``w_ptr_a`` / ``w_ptr_b``: int64
+    ``[1, num_experts]`` bank-address tables (:func:`fill_w_ptr`), A_down[l, e] being the
+    ``[rank, I]`` row-major block ``l * lora_stride_a`` elements into expert e's A bank and
+    B_down[l, e] the ``[H, rank]`` block ``l * lora_stride_b`` elements into its B bank.  The banks
+    must live on the activation's device; adapter ids must exist in them.  Routing entries are
+    read on the device: one out of range is skipped and :func:`nvfp4lora_device_status` raises
+    ValueError."""
+    act = gemm1_activation_output
+    if lora_dtype not in _DTYPE_CODES or out_dtype not in _DTYPE_CODES:
+        raise ValueError("lora_dtype and out_dtype must be torch.bfloat16 or torch.float16")
+    _need(act, "gemm1_activation_output", lora_dtype, 2)
+    _need(expanded_idx_to_permuted_idx, "expanded_idx_to_permuted_idx", torch.int32)
+    _need(w_ptr_a, "w_ptr_a", torch.int64)
+    _need(w_ptr_b, "w_ptr_b", torch.int64)
+    _need(topk_ids, "topk_ids", torch.int32, 2)
+    _need(topk_weights, "topk_weights", torch.float32, 2)
+    _need(lora_ids, "lora_ids", torch.int32, 1)
+    T, top_k = topk_ids.shape
+    E = w_ptr_a.numel()
+    if w_ptr_b.numel() != E:
+        raise ValueError(f"w_ptr_a has {E} entries but w_ptr_b has {w_ptr_b.numel()}")
+    if tuple(topk_weights.shape) != (T, top_k) or lora_ids.shape[0] != T:
+        raise ValueError(f"topk_weights must be [T, top_k] = [{T}, {top_k}] and lora_ids [T]")
+    if expanded_idx_to_permuted_idx.numel() != T * top_k:
+        raise ValueError(f"expanded_idx_to_permuted_idx must hold T * top_k = {T * top_k} entries")
+    H = int(hidden_size)
+    if out is None:
+        out = torch.empty((T, H), dtype=out_dtype, device=act.device)
+    else:
+        _need(out, "out", out_dtype, 2)
+        if tuple(out.shape) != (T, H):
+            raise ValueError(f"out must be [T, hidden_size] = [{T}, {H}]")
+    _same_device("gemm1_activation_output", act, expanded_idx_to_permuted_idx=expanded_idx_to_permuted_idx,
+                 w_ptr_a=w_ptr_a, w_ptr_b=w_ptr_b, topk_ids=topk_ids, topk_weights=topk_weights, lora_ids=lora_ids,
+                 out=out)
+    with torch.cuda.device(act.device):
+        nvfp4lora_bgmv_moe_gemm2_lora_delta(act, act.shape[0], act.shape[1], expanded_idx_to_permuted_idx, w_ptr_a,
+                                            lora_stride_a, w_ptr_b, lora_stride_b, topk_ids, topk_weights, lora_ids,
+                                            T, top_k, E, rank, H, _DTYPE_CODES[lora_dtype], scale,
+                                            _DTYPE_CODES[out_dtype], out, torch.cuda.current_stream(act.device))
     return out
 
 

@@ -22,6 +22,7 @@
 #include <string>
 
 #include "../../include/nvfp4lora.h"
+#include "bgmv.cuh"
 #include "fold.cuh"
 #include "gemm.cuh"
 #include "gemm_decode.cuh"
@@ -92,13 +93,13 @@ nvfp4lora_status device_info(int* dev_out, DeviceInfo** info_out) {
 }
 
 template <typename Kernel>
-nvfp4lora_status ensure_smem_attr(DeviceInfo* info, Kernel kernel, int smem) {
+nvfp4lora_status ensure_smem_attr(DeviceInfo* info, Kernel kernel, int smem, bool max_carveout = true) {
     std::lock_guard<std::mutex> lock(g_mu);
     const void* key = reinterpret_cast<const void*>(kernel);
     if (info->smem_attr_set.count(key)) return NVFP4LORA_OK;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     // the whole unified L1 / shared array as shared memory, so co-resident CTAs fit
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && max_carveout)
         e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     info->smem_attr_set.insert(key);
@@ -834,6 +835,11 @@ nvfp4lora_status nvfp4lora_device_status(nvfp4lora_stream stream) {
             return fail(NVFP4LORA_ERR_INVALID_ARG,
                         "grouped call: m_indptr must start at 0, be non-decreasing, hold multiples of 128 and "
                         "end at most at the row count (no tile was computed)");
+        if (word == kErrBadRoute)
+            return fail(NVFP4LORA_ERR_INVALID_ARG,
+                        "LoRA delta: a routing entry was out of range (expert id outside [0, num_experts), "
+                        "permuted index past the activation rows, or a null or misaligned bank address); "
+                        "that slot was skipped");
         return fail(NVFP4LORA_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (pipeline stalled)");
     }
     return NVFP4LORA_OK;
@@ -884,6 +890,120 @@ nvfp4lora_status nvfp4lora_quantize(const uint16_t* x, int64_t rows, int64_t K, 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
     return NVFP4LORA_OK;
+}
+
+nvfp4lora_status nvfp4lora_bgmv_moe_gemm2_lora_delta(
+    const void* act, int64_t padded_rows, int64_t I, const int32_t* perm, const int64_t* w_ptr_a,
+    int64_t lora_stride_a, const int64_t* w_ptr_b, int64_t lora_stride_b, const int32_t* topk_ids,
+    const float* topk_weights, const int32_t* lora_ids, int64_t num_tokens, int64_t top_k, int64_t num_experts,
+    int64_t rank, int64_t hidden_size, int32_t lora_dtype, float scale, int32_t out_dtype, void* out,
+    nvfp4lora_stream stream) {
+    t_last_error.clear();
+    const int64_t kMaxDim = (int64_t)1 << 30;
+    if (num_tokens < 0 || num_tokens > kMaxDim)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "num_tokens = %lld out of range", (long long)num_tokens);
+    if (top_k < 1 || top_k > kBgmvMaxTopK)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "top_k = %lld: 1 <= top_k <= %d is required", (long long)top_k,
+                    kBgmvMaxTopK);
+    if (rank < 8 || rank > kBgmvMaxRank || rank % 8 != 0)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "rank = %lld: 8 <= rank <= %d with rank %% 8 == 0 is required",
+                    (long long)rank, kBgmvMaxRank);
+    if (I < 8 || I % 8 != 0 || I > kMaxDim)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "I = %lld: I >= 8 with I %% 8 == 0 is required", (long long)I);
+    if (hidden_size < 1 || hidden_size > kMaxDim)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "hidden_size = %lld out of range", (long long)hidden_size);
+    if (num_experts < 1 || num_experts > kMaxDim)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "num_experts = %lld out of range", (long long)num_experts);
+    if (padded_rows < 0 || padded_rows > kMaxDim)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "padded_rows = %lld out of range", (long long)padded_rows);
+    if (num_tokens * top_k > kMaxDim)
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "num_tokens * top_k too large");
+    if (lora_stride_a < 0 || lora_stride_b < 0 || lora_stride_a % 8 != 0 || lora_stride_b % 8 != 0)
+        return fail(NVFP4LORA_ERR_INVALID_ARG,
+                    "lora_stride_a = %lld, lora_stride_b = %lld: non-negative multiples of 8 are required "
+                    "(adapter blocks start on 16-byte boundaries)", (long long)lora_stride_a, (long long)lora_stride_b);
+    if ((lora_dtype != NVFP4LORA_DTYPE_BF16 && lora_dtype != NVFP4LORA_DTYPE_FP16) ||
+        (out_dtype != NVFP4LORA_DTYPE_BF16 && out_dtype != NVFP4LORA_DTYPE_FP16))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "lora_dtype and out_dtype must be NVFP4LORA_DTYPE_BF16 or _FP16");
+    if (num_tokens == 0) return NVFP4LORA_OK;
+    if (!perm || !w_ptr_a || !w_ptr_b || !topk_ids || !topk_weights || !lora_ids || !out ||
+        (!act && padded_rows > 0))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "every pointer argument must be non-null");
+    if (!aligned(act, 16)) return fail(NVFP4LORA_ERR_INVALID_ARG, "act must be 16-byte aligned");
+    if (!aligned(w_ptr_a, 8) || !aligned(w_ptr_b, 8))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "w_ptr_a and w_ptr_b must be 8-byte aligned");
+    if (!aligned(perm, 4) || !aligned(topk_ids, 4) || !aligned(topk_weights, 4) || !aligned(lora_ids, 4) ||
+        !aligned(out, 2))
+        return fail(NVFP4LORA_ERR_INVALID_ARG, "routing tables must be 4-byte aligned and out 2-byte aligned");
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    nvfp4lora_status st = device_info(&dev, &info);
+    if (st != NVFP4LORA_OK) return st;
+
+    // A cluster of cs CTAs per token splits I (shrink) and H (expand): the smallest power of two
+    // that gives about two CTAs per SM, capped by the cluster limit and by I / 8 and H; raised
+    // further if one CTA's shared memory (the shrink's cells for its I slice) would not fit.
+    const int64_t len = top_k * rank;
+    auto fits = [&](int64_t c) { return bgmv_smem_floats(len, (I / 8 + c - 1) / c, c) * 4 <= kBgmvSmemLimit; };
+    auto can_grow = [&](int64_t c) { return c < kBgmvMaxCluster && 2 * c <= I / 8 && 2 * c <= hidden_size; };
+    int cs = 1;
+    while (can_grow(cs) && num_tokens * cs < 2 * (int64_t)info->sms) cs *= 2;
+    while (!fits(cs) && can_grow(cs)) cs *= 2;
+    if (!fits(cs))
+        return fail(NVFP4LORA_ERR_INVALID_ARG,
+                    "top_k * rank * I too large: one CTA's share (I / %d columns, %lld rows of the adapters) needs more "
+                    "than %d bytes of shared memory", cs, (long long)len, kBgmvSmemLimit);
+    BgmvArgs args;
+    args.act = act;
+    args.perm = perm;
+    args.w_ptr_a = w_ptr_a;
+    args.w_ptr_b = w_ptr_b;
+    args.topk_ids = topk_ids;
+    args.topk_w = topk_weights;
+    args.lora_ids = lora_ids;
+    args.out = out;
+    args.stride_a = lora_stride_a;
+    args.stride_b = lora_stride_b;
+    args.rows = (int)padded_rows;
+    args.I = (int)I;
+    args.top_k = (int)top_k;
+    args.num_experts = (int)num_experts;
+    args.rank = (int)rank;
+    args.H = (int)hidden_size;
+    args.cs = cs;
+    args.scale = scale;
+    const int smem = (int)(bgmv_smem_floats(len, (I / 8 + cs - 1) / cs, cs) * (int64_t)sizeof(float));
+
+    auto pick = [&](auto kernel) -> nvfp4lora_status {
+        // the delta's shared memory can exceed the 48 KB default; the L1 carve-out stays the
+        // driver's choice (the activation rows are re-read through L1)
+        nvfp4lora_status sa = ensure_smem_attr(info, kernel, kBgmvSmemLimit, false);
+        if (sa != NVFP4LORA_OK) return sa;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(num_tokens * cs));
+        cfg.blockDim = dim3(kBgmvThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cs > 1) {
+            attr[1].id = cudaLaunchAttributeClusterDimension;
+            attr[1].val.clusterDim.x = cs;
+            attr[1].val.clusterDim.y = 1;
+            attr[1].val.clusterDim.z = 1;
+            cfg.numAttrs = 2;
+        }
+        cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args);
+        if (e != cudaSuccess) return cuda_fail(e, "LoRA delta launch");
+        return NVFP4LORA_OK;
+    };
+    const bool f16_in = lora_dtype == NVFP4LORA_DTYPE_FP16, f16_out = out_dtype == NVFP4LORA_DTYPE_FP16;
+    if (f16_in)
+        return f16_out ? pick(bgmv_delta_kernel<true, true>) : pick(bgmv_delta_kernel<true, false>);
+    return f16_out ? pick(bgmv_delta_kernel<false, true>) : pick(bgmv_delta_kernel<false, false>);
 }
 
 const char* nvfp4lora_last_error(void) { return t_last_error.c_str(); }

@@ -170,3 +170,48 @@ def test_grouped_rules_are_checked_before_cuda(lib):
                       (dict(a_sf_bytes=512 * 16 - 1), b"a_sf")):
         assert call(**bad) == 1, bad
         assert word in lib.nvfp4lora_last_error(), (bad, lib.nvfp4lora_last_error())
+
+
+def test_lora_delta_rules_are_checked_before_cuda(lib):
+    f = lib.nvfp4lora_bgmv_moe_gemm2_lora_delta
+    f.restype = ctypes.c_int
+    f.argtypes = [P, I64, I64, P, P, I64, P, I64, P, P, P, I64, I64, I64, I64, I64, ctypes.c_int32, ctypes.c_float,
+                  ctypes.c_int32, P, P]
+    lib.nvfp4lora_last_error.restype = ctypes.c_char_p
+    ok = dict(act=0x10000, rows=256, I=512, perm=0x20000, wa=0x30000, sa=16 * 512, wb=0x40000, sb=256 * 16,
+              ids=0x50000, w=0x60000, lids=0x70000, T=8, top_k=2, E=4, rank=16, H=256, ldt=0, scale=1.0, odt=0,
+              out=0x80000)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["act"], a["rows"], a["I"], a["perm"], a["wa"], a["sa"], a["wb"], a["sb"], a["ids"], a["w"],
+                 a["lids"], a["T"], a["top_k"], a["E"], a["rank"], a["H"], a["ldt"], a["scale"], a["odt"], a["out"],
+                 None)
+
+    for bad, word in ((dict(rank=12), b"rank"), (dict(rank=136), b"rank"), (dict(top_k=0), b"top_k"),
+                      (dict(top_k=17), b"top_k"), (dict(I=100), b"I = 100"), (dict(H=0), b"hidden_size"),
+                      (dict(E=0), b"num_experts"), (dict(sa=12), b"lora_stride"), (dict(sb=-8), b"lora_stride"),
+                      (dict(ldt=2), b"dtype"), (dict(odt=-1), b"dtype"), (dict(T=-1), b"num_tokens"),
+                      (dict(perm=None), b"non-null"), (dict(out=None), b"non-null"),
+                      (dict(act=0x10008), b"16-byte"), (dict(wa=0x30004), b"8-byte"),
+                      (dict(ids=0x50002), b"4-byte")):
+        assert call(**bad) == 1, bad
+        assert word in lib.nvfp4lora_last_error(), (bad, lib.nvfp4lora_last_error())
+    # no tokens: nothing to do, and nothing is enqueued (no CUDA call is made)
+    assert call(T=0, perm=None, out=None) == 0
+
+
+def test_lora_delta_binding_rules():
+    import torch
+    import nvfp4_block_scaled_mm_b200 as L
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        L.fill_w_ptr([torch.zeros(4, dtype=torch.bfloat16)])
+    with pytest.raises(ValueError, match="at least one"):
+        L.fill_w_ptr([])
+    with pytest.raises(ValueError, match="lora_dtype"):
+        L.bgmv_moe_gemm2_lora_delta(torch.zeros(1, 8), None, None, 0, None, 0, None, None, None, 8, 8,
+                                    lora_dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        L.bgmv_moe_gemm2_lora_delta(torch.zeros(1, 8, dtype=torch.bfloat16), None, None, 0, None, 0, None, None,
+                                    None, 8, 8)
