@@ -91,3 +91,34 @@ def test_grouped_moe_shape_sampled():
                                      rng.choice(int(ind[-1]), 96, replace=False)]))
     y = oracle(p, 0.5)
     check_close(out[torch.from_numpy(rows).cuda()], y[rows], what="moe sampled rows")
+
+
+def test_grouped_graph_replay_with_new_routing():
+    """m_indptr is read on the device only, so one captured grouped call serves a new expert split
+    copied into its captured table (same total row count here, different segments)."""
+    dev = "cuda"
+    p1 = make_grouped_problem([256, 128, 0, 128], 264, 512, 16, seed=51, pad_rows=128)
+    p2 = make_grouped_problem([128, 0, 384, 0], 264, 512, 16, seed=51, pad_rows=128)
+    assert p1.rows == p2.rows
+    t = {k: getattr(p1, k).to(dev) for k in ("m_indptr", "a", "b", "a_sf", "b_sf", "alpha", "d", "lora_b")}
+    bias = p1.bias.to(dev)
+    s = torch.tensor([1.25], dtype=torch.float32, device=dev)
+    out = torch.full((p1.rows, p1.N), 1.0, dtype=torch.bfloat16, device=dev)
+
+    def call():
+        L.grouped_mm_nvfp4_lora(t["a"], t["b"], t["a_sf"], t["b_sf"], t["m_indptr"], t["alpha"], t["d"],
+                                t["lora_b"], s, bias=bias, out=out)
+
+    call()                                   # warm-up outside the capture
+    L.nvfp4lora_device_status()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    # the same operands (drawn with the same seed), a different split of the rows among the experts
+    t["m_indptr"].copy_(p2.m_indptr.to(dev))
+    out.fill_(1.0)
+    graph.replay()
+    L.nvfp4lora_device_status()
+    used = int(p2.m_indptr[-1])
+    check_close(out[:used], oracle(p2, 1.25), what="grouped graph replay")
+    assert torch.all(out[used:].view(torch.int16) == SENTINEL)
