@@ -65,6 +65,8 @@ SHAPES = [
     (1, 1, 2, 2, 4096, 4096, 128, BF, HF, 0, 128),    # one token, rank 128, clusters of 8
     (64, 2, 8, 4, 4096, 4096, 16, HF, BF, 0, 128),    # the decode batch, fp16 in, bf16 out
     (150, 16, 32, 2, 256, 512, 8, BF, BF, 8, 8),      # top_k 16
+    (24, 16, 20, 2, 1024, 520, 128, BF, BF, 0, 16),   # the largest slot set: top_k 16 x rank 128, clusters
+    (320, 16, 20, 2, 1024, 264, 128, HF, BF, 8, 128),  # the same with one CTA per token
 ]
 
 

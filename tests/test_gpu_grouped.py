@@ -122,3 +122,16 @@ def test_grouped_graph_replay_with_new_routing():
     used = int(p2.m_indptr[-1])
     check_close(out[:used], oracle(p2, 1.25), what="grouped graph replay")
     assert torch.all(out[used:].view(torch.int16) == SENTINEL)
+
+
+def test_grouped_maximum_expert_count():
+    """511 experts (the limit), most of them empty: the device-side table copy and the binary search
+    over all 512 entries, with non-empty experts at both ends and in the middle."""
+    segments = [0] * 511
+    for e in (0, 255, 510):
+        segments[e] = 128
+    p = make_grouped_problem(segments, 136, 256, 8, seed=77, pad_rows=0)
+    assert p.m_indptr.numel() == 512
+    out = run(p, 0.75)
+    L.nvfp4lora_device_status()
+    check_close(out, oracle(p, 0.75), what="grouped, 511 experts")
