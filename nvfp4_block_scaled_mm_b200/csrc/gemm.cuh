@@ -78,7 +78,10 @@ constexpr int kTileN = 256;
 constexpr int kEpiWarps = 8;
 constexpr int kOutBoxCols = 32;          // TMA store box of the epilogue: 32 columns x 32 rows
 constexpr int kOutBoxRows = 32;
-constexpr int kOutBoxes = 3;             // per epilogue warp: a box is rewritten once its store has read it
+// Output staging: one 32 x 32 box per epilogue warp, rewritten once its previous store has read it
+// (the epilogue has slack).  Against three boxes: the 8-expert grouped layer 37.5 us per call
+// against 38.8, the M = 64 and 96 calls within 1 %.
+constexpr int kOutBoxes = 1;
 constexpr int kSfStages = 4;             // scale-atom ring (own barriers, recycled by the staging warps)
 constexpr int kGemmThreads = 512;        // 4 warpgroups: producers/MMA, staging, 2 x epilogue
 // Registers per thread after the split.  The block is launched with 512 x 128; the split must not
