@@ -488,17 +488,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 if (!__all_sync(kAll, mbar_wait(&sf_full[sst], sphase, abort_flag))) { ok = false; break; }
                 const uint8_t* srca = smem + L::SFA_OFF + sst * L::SFA_BYTES + lane * 16;
                 const uint8_t* srcb = smem + L::SFB_OFF + sst * L::SFB_BYTES + lane * 16;
-                uint32_t va[16], vb[32];
+                uint32_t va[16];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint4 w = *reinterpret_cast<const uint4*>(srca + j * 512);
                     va[4 * j] = w.x; va[4 * j + 1] = w.y; va[4 * j + 2] = w.z; va[4 * j + 3] = w.w;
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(srcb + j * 512);
-                    const uint4 w1 = *reinterpret_cast<const uint4*>(srcb + 2048 + j * 512);
-                    vb[8 * j] = w0.x; vb[8 * j + 1] = w0.y; vb[8 * j + 2] = w0.z; vb[8 * j + 3] = w0.w;
-                    vb[8 * j + 4] = w1.x; vb[8 * j + 5] = w1.y; vb[8 * j + 6] = w1.z; vb[8 * j + 7] = w1.w;
                 }
-                // the slot's previous MMAs have completed (its loads overlap this wait)
+                // the slot's previous MMAs have completed (the A loads overlap this wait; the B atoms
+                // are read after it, which keeps the warp within its 72 registers)
                 if (use > 0 && !__all_sync(kAll, mbar_wait(&slot_free[slot], (use - 1) & 1u, abort_flag))) {
                     ok = false;
                     break;
@@ -506,6 +503,14 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
                 tc_fence_after();
                 const uint32_t col = tmem + lane_off + T::SF0 + slot * T::SLOT_COLS;
                 tmem_store_16(col, va);
+                uint32_t vb[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(srcb + j * 512);
+                    const uint4 w1 = *reinterpret_cast<const uint4*>(srcb + 2048 + j * 512);
+                    vb[8 * j] = w0.x; vb[8 * j + 1] = w0.y; vb[8 * j + 2] = w0.z; vb[8 * j + 3] = w0.w;
+                    vb[8 * j + 4] = w1.x; vb[8 * j + 5] = w1.y; vb[8 * j + 6] = w1.z; vb[8 * j + 7] = w1.w;
+                }
                 tmem_store_32(col + T::SFA_COLS, vb);
                 // the stores have read their registers, so the loads are done: the ring slot is free
                 __syncwarp();
