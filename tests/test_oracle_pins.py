@@ -724,3 +724,32 @@ def test_f16_rounding_against_numpy_and_hand_cases():
     assert got[-10] == 0x3C00 and got[-9] == 0x3C02          # ties to even at 1
     assert got[-6] == 0x7BFF and got[-5] == 0x7C00 and got[-4] == 0xFC00
     assert got[-3] == 0x0000 and got[-1] == 0x8000             # half the smallest subnormal -> 0
+
+
+def test_bgmv_generator_routing_layout():
+    """The LoRA-delta input generator lays the routed slots out as the recipe states: each token's
+    experts distinct, weights positive and summing to 1, every active slot's row inside its expert's
+    segment, segments ordered by expert and padded to the alignment, stride padding NaN."""
+    import workloads as W
+    p = W.make_bgmv_problem(40, 4, 6, 3, 64, 32, 8, seed=13, stride_pad=8, seg_align=16, p_inactive=0.1)
+    ids = p.topk_ids.numpy()
+    assert all(len(set(row)) == p.top_k for row in ids)
+    w = p.topk_weights.numpy()
+    assert np.all(w > 0) and np.allclose(w.sum(axis=1), 1.0, atol=1e-6)
+    perm = p.perm.numpy().reshape(p.T, p.top_k)
+    rows_of = {e: [] for e in range(p.num_experts)}
+    for t in range(p.T):
+        for j in range(p.top_k):
+            if perm[t, j] >= 0:
+                rows_of[int(ids[t, j])].append(int(perm[t, j]))
+    used = [r for e in rows_of for r in rows_of[e]]
+    assert len(used) == len(set(used)), "two slots share an activation row"
+    start = 0
+    for e in range(p.num_experts):
+        n = int((ids == e).sum())
+        seg = -(-n // 16) * 16
+        assert all(start <= r < start + seg for r in rows_of[e])
+        start += seg
+    assert p.act.shape[0] >= start
+    bank = p.a_banks[0].float().numpy().reshape(p.num_adapters, p.stride_a)
+    assert np.all(np.isnan(bank[:, p.rank * p.I:])) and not np.any(np.isnan(bank[:, :p.rank * p.I]))
