@@ -302,8 +302,10 @@ def test_zero_adapter_bitwise(M, N, K, r):
 # padding rows of the scale buffers never reach rows < M or columns < N
 # ---------------------------------------------------------------------------------------
 
-def test_nan_poisoned_scale_padding():
-    M, N, K, r = 16, 200, 512, 16
+@pytest.mark.parametrize("M,N", [(16, 200), (20, 136), (70, 200), (200, 300)],
+                         ids=["decode16", "decode32", "single_sm", "sm_pair"])
+def test_nan_poisoned_scale_padding(M, N):
+    K, r = 512, 16
     p = make_problem(M, N, K, r, seed=8, alpha=2.0 ** -6, lora_scale=1.0, bias=True)
     for buf, rows in ((p.a_sf, M), (p.b_sf, N)):
         rp = -(-rows // 128) * 128
