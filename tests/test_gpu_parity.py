@@ -174,7 +174,9 @@ SHAPES = [(1, 8, 256, 8), (16, 4096, 256, 64), (200, 300, 512, 16), (130, 1000, 
           (3, 256, 2048, 16), (32, 1000, 1024, 128), (20, 9000, 512, 8), (16, 4096, 4096, 64),
           (33, 520, 512, 40), (600, 520, 512, 24), (513, 256, 256, 8), (64, 300, 512, 16),
           (100, 1000, 768, 72), (127, 520, 1024, 8), (200, 600, 512, 8), (256, 1000, 768, 24),
-          (256, 520, 512, 40)]
+          (256, 520, 512, 40),
+          # a single output column and three (outputs of 2 and 6 bytes per row: the plain-store path)
+          (1, 1, 256, 8), (40, 3, 512, 8), (130, 1, 256, 16)]
 
 
 @pytest.mark.parametrize("M,N,K,r", SHAPES)
